@@ -1,0 +1,322 @@
+/*
+ * bitnet_oracle.c -- the plain, slow CPU definition of the H-BitLinear forward path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may load this file or
+ * the library built from it: only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with the
+ * CUDA library; the only thing both sides see is the seeded synthetic inputs.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC (see build.py in
+ * this folder).  -ffp-contract=off keeps every a*b+c as two IEEE roundings, so
+ * each fp32 expression below means exactly what it says.  Single-threaded.
+ *
+ * Sources (page titles as given on the pages):
+ *   [v2]   "bitnet_v2_engine.py" (Quillan-Ronin colab bundle): the BitNet v2
+ *          restatement, Eq. 1-7 in its module docstring, fast_hadamard_transform,
+ *          quantize_weight_ternary, quantize_act_int8, quantize_act_int4,
+ *          HBitLinear.forward.
+ *   [b158] "BitNet 论文解析" (youngju.dev transcription), section on BitNet b1.58:
+ *          weight_quant_ternary and the integer-GEMM + rescale form of
+ *          BitLinear_b158.forward; the {-1,0,+1} -> {0,1,2} code map of its
+ *          tl2_lookup_simulation listing.
+ *   [edge] "bitnet_cpp_edge.py": pack-once / forward-many (prepare_weights) and the
+ *          claim that per-token integer kernels are lossless.
+ *
+ * Readings where the pages are silent or disagree (each one is listed in the
+ * design notes with its reason):
+ *   - eps = 1e-5 is passed in by the caller (the pages use 1e-7 and 1e-5).
+ *   - Rounding is round-half-to-even (the pages call torch.round).
+ *   - RMSNorm is y = (x * r) * g with r = 1 / sqrt(sum(x^2)/K + eps).
+ *   - The FWHT scales every butterfly stage by c = (float)(1/sqrt 2), as the
+ *     listing of fast_hadamard_transform does, in natural (Sylvester) order.
+ *   - The per-token scale returned is gamma (or beta) without eps (Eq. 5/6).
+ *   - alpha = mean|W| is summed in double in index order, rounded once to float.
+ *   - The dequant epilogue is out = (float)acc * ((alpha * scale_x) / Q).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_ACT_INT8 0
+#define ORACLE_ACT_INT4 1
+
+/* return codes */
+#define ORACLE_OK 0
+#define ORACLE_NOT_POW2 3
+#define ORACLE_BAD_ARG 1
+
+static float q_int8(void) { return 127.0f; }
+static float q_int4(void) { return (float)sqrt(7.0); } /* sqrt(7) rounded once to float */
+
+static int is_pow2(int64_t n) { return n > 0 && (n & (n - 1)) == 0; }
+
+/* Round to nearest, ties to even, in the current (default) rounding mode. */
+static float rne(float v) { return nearbyintf(v); }
+
+static float clampf(float v, float lo, float hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+/* ---------------------------------------------------------------------------
+ * Step 1. RMSNorm, per token.  [v2] HBitLinear.forward "Normalization" (the page
+ * builds nn.RMSNorm(in_features, eps) but does not define it; this is the usual
+ * root-mean-square normalisation with a per-channel gain).
+ *   ss  = sum_k x[k]*x[k]        (fp32, k ascending)
+ *   r   = 1 / sqrt(ss/K + eps)   (IEEE sqrt and division)
+ *   y_k = (x_k * r) * g_k        (g == NULL means g = 1)
+ * ------------------------------------------------------------------------- */
+int oracle_rmsnorm(const float *x, int64_t M, int64_t K, const float *g, float eps,
+                   float *y)
+{
+    if (K <= 0 || M < 0) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xr = x + m * K;
+        float *yr = y + m * K;
+        float ss = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float sq = xr[k] * xr[k];
+            ss = ss + sq;
+        }
+        float mean = ss / (float)K;
+        float r = 1.0f / sqrtf(mean + eps);
+        for (int64_t k = 0; k < K; ++k) {
+            float v = xr[k] * r;
+            yr[k] = g ? v * g[k] : v;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 2. Fast Walsh-Hadamard transform along each row, in place.
+ * [v2] Eq. 3/4: H_m = (1/sqrt 2) [[H_{m-1}, H_{m-1}], [H_{m-1}, -H_{m-1}]], H_0 = [1];
+ * fast_hadamard_transform: radix-2 butterflies with half-width h = 1, 2, 4, ...,
+ * each stage scaled by 1/sqrt 2, computed in fp32.  K must be a power of two
+ * (the page raises ValueError otherwise; here the call returns ORACLE_NOT_POW2).
+ * ------------------------------------------------------------------------- */
+int oracle_fwht(float *y, int64_t M, int64_t K)
+{
+    if (!is_pow2(K)) return ORACLE_NOT_POW2;
+    const float c = (float)(1.0 / sqrt(2.0));
+    for (int64_t m = 0; m < M; ++m) {
+        float *row = y + m * K;
+        for (int64_t h = 1; h < K; h *= 2) {
+            for (int64_t j0 = 0; j0 < K; j0 += 2 * h) {
+                for (int64_t j = j0; j < j0 + h; ++j) {
+                    float u = row[j];
+                    float v = row[j + h];
+                    row[j] = (u + v) * c;
+                    row[j + h] = (u - v) * c;
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 3. Per-token activation quantisation.
+ * int8 absmax  [v2] Eq. 5: gamma = max|y|,  q = RoundClip(127 * y / (gamma+eps), -128, 127)
+ * int4 absmean [v2] Eq. 6: beta  = mean|y|, q = RoundClip(sqrt7 * y / (beta+eps),  -8,   7)
+ * The listings form the per-token multiplier first, s = Q / (gamma + eps), and then
+ * multiply: q = clamp(rne(y * s)).  scale_x[m] = gamma (or beta), without eps.
+ * ------------------------------------------------------------------------- */
+int oracle_act_quant(const float *y, int64_t M, int64_t K, int mode, float eps,
+                     int8_t *q, float *scale_x)
+{
+    if (K <= 0 || M < 0) return ORACLE_BAD_ARG;
+    if (mode != ORACLE_ACT_INT8 && mode != ORACLE_ACT_INT4) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const float *yr = y + m * K;
+        int8_t *qr = q + m * K;
+        float stat, s, lo, hi;
+        if (mode == ORACLE_ACT_INT8) {
+            float gamma = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                float a = fabsf(yr[k]);
+                if (a > gamma) gamma = a;
+            }
+            stat = gamma;
+            s = q_int8() / (gamma + eps);
+            lo = -128.0f;
+            hi = 127.0f;
+        } else {
+            float sum = 0.0f;
+            for (int64_t k = 0; k < K; ++k) sum = sum + fabsf(yr[k]);
+            float beta = sum / (float)K;
+            stat = beta;
+            s = q_int4() / (beta + eps);
+            lo = -8.0f;
+            hi = 7.0f;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            float v = yr[k] * s;
+            qr[k] = (int8_t)clampf(rne(v), lo, hi);
+        }
+        scale_x[m] = stat;
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * fp64 shadow of steps 1-3: the pre-rounding value y*s of every code, with every
+ * step carried in double (the FWHT as the same butterflies in double).  Tests use
+ * it to tell a rounding near-tie, where two correct fp32 evaluation orders may
+ * land on different codes, from a real disagreement.
+ * ------------------------------------------------------------------------- */
+int oracle_shadow_prerounding(const float *x, int64_t M, int64_t K, const float *g,
+                              double eps, int fwht, int mode, double *v)
+{
+    if (K <= 0 || M < 0) return ORACLE_BAD_ARG;
+    if (fwht && !is_pow2(K)) return ORACLE_NOT_POW2;
+    double *row = (double *)malloc((size_t)K * sizeof(double));
+    if (!row) return ORACLE_BAD_ARG;
+    const double c = 1.0 / sqrt(2.0);
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xr = x + m * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) ss += (double)xr[k] * (double)xr[k];
+        double r = 1.0 / sqrt(ss / (double)K + eps);
+        for (int64_t k = 0; k < K; ++k) row[k] = (double)xr[k] * r * (g ? (double)g[k] : 1.0);
+        if (fwht) {
+            for (int64_t h = 1; h < K; h *= 2)
+                for (int64_t j0 = 0; j0 < K; j0 += 2 * h)
+                    for (int64_t j = j0; j < j0 + h; ++j) {
+                        double a = row[j], b = row[j + h];
+                        row[j] = (a + b) * c;
+                        row[j + h] = (a - b) * c;
+                    }
+        }
+        double s;
+        if (mode == ORACLE_ACT_INT8) {
+            double gamma = 0.0;
+            for (int64_t k = 0; k < K; ++k) gamma = fabs(row[k]) > gamma ? fabs(row[k]) : gamma;
+            s = 127.0 / (gamma + eps);
+        } else {
+            double sum = 0.0;
+            for (int64_t k = 0; k < K; ++k) sum += fabs(row[k]);
+            s = sqrt(7.0) / (sum / (double)K + eps);
+        }
+        for (int64_t k = 0; k < K; ++k) v[m * K + k] = row[k] * s;
+    }
+    free(row);
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 4a. Ternary weights, per tensor.  [v2] Eq. 1/2, quantize_weight_ternary;
+ * [b158] weight_quant_ternary.
+ *   alpha = mean|W|   (summed in double, index order, one rounding to float)
+ *   t     = RoundClip(W / (alpha + eps), -1, 1)   (fp32 division)
+ * ------------------------------------------------------------------------- */
+float oracle_weight_alpha(const float *W, int64_t count)
+{
+    double sum = 0.0;
+    for (int64_t i = 0; i < count; ++i) sum += fabs((double)W[i]);
+    return (float)(sum / (double)count);
+}
+
+int oracle_ternarize(const float *W, int64_t count, float alpha, float eps, int8_t *t)
+{
+    float d = alpha + eps;
+    for (int64_t i = 0; i < count; ++i) {
+        float v = W[i] / d;
+        t[i] = (int8_t)clampf(rne(v), -1.0f, 1.0f);
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 4b. 2-bit packing of the ternary codes (layout fixed by the library
+ * header; restated here from that document, not shared with it).
+ * Code map [b158] tl2_lookup_simulation: -1 -> 0, 0 -> 1, +1 -> 2 (3 is never
+ * written).  packed is [N][K/4] bytes, row n starting at byte n*K/4.  Inside a row,
+ * k = 16*w + 4*j + b (w = k/16, j = (k%16)/4, b = k%4) lives in byte 4*w + b,
+ * bits [2j, 2j+2).  K must be a multiple of 16.
+ * ------------------------------------------------------------------------- */
+int oracle_pack(const int8_t *t, int64_t N, int64_t K, uint8_t *packed)
+{
+    if (K <= 0 || K % 16 != 0 || N < 0) return ORACLE_BAD_ARG;
+    const int64_t row_bytes = K / 4;
+    memset(packed, 0, (size_t)(N * row_bytes));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int v = t[n * K + k];
+            if (v < -1 || v > 1) return ORACLE_BAD_ARG;
+            unsigned code = (unsigned)(v + 1);
+            int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
+            packed[n * row_bytes + 4 * w + b] |= (uint8_t)(code << (2 * j));
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *t)
+{
+    if (K <= 0 || K % 16 != 0 || N < 0) return ORACLE_BAD_ARG;
+    const int64_t row_bytes = K / 4;
+    int bad = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
+            unsigned code = (packed[n * row_bytes + 4 * w + b] >> (2 * j)) & 3u;
+            if (code == 3u) bad = 1;
+            t[n * K + k] = (int8_t)((int)code - 1);
+        }
+    }
+    return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 5. Integer GEMM of activation codes with ternary weights.
+ * [v2] HBitLinear.forward: F.linear(x_q, w_q), i.e. out[m][n] = sum_k x[m][k] W[n][k];
+ * [b158] BitLinear_b158.forward does it on the integer codes and rescales after.
+ *   acc[m][n] = sum_k q[m][k] * t[n][k]    (exact in int32: |acc| <= 128*K)
+ * The packed variant reads each weight code straight out of the packed bytes.
+ * ------------------------------------------------------------------------- */
+int oracle_gemm_int(const int8_t *q, const int8_t *t, int64_t M, int64_t N, int64_t K,
+                    int32_t *acc)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k) s += (int32_t)q[m * K + k] * (int32_t)t[n * K + k];
+            acc[m * N + n] = s;
+        }
+    return ORACLE_OK;
+}
+
+int oracle_gemm_packed(const int8_t *q, const uint8_t *packed, int64_t M, int64_t N,
+                       int64_t K, int32_t *acc)
+{
+    if (K <= 0 || K % 16 != 0) return ORACLE_BAD_ARG;
+    const int64_t row_bytes = K / 4;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
+                int code = (packed[n * row_bytes + 4 * w + b] >> (2 * j)) & 3;
+                s += (int32_t)q[m * K + k] * (int32_t)(code - 1);
+            }
+            acc[m * N + n] = s;
+        }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Step 6. Dequant epilogue.  The forward's F.linear of the two dequantised
+ * operands equals acc * alpha * scale_x / Q ([b158]: output*(w_scale*x_scale)/Qb;
+ * [v2] Eq. 5/6 give gamma/127 and beta/sqrt7 as the activation step sizes).
+ *   f_m = (alpha * scale_x[m]) / Q ;  out[m][n] = (float)acc[m][n] * f_m
+ * ------------------------------------------------------------------------- */
+int oracle_dequant(const int32_t *acc, const float *scale_x, float alpha, int mode,
+                   int64_t M, int64_t N, float *out)
+{
+    if (mode != ORACLE_ACT_INT8 && mode != ORACLE_ACT_INT4) return ORACLE_BAD_ARG;
+    const float Q = mode == ORACLE_ACT_INT8 ? q_int8() : q_int4();
+    for (int64_t m = 0; m < M; ++m) {
+        float f = (alpha * scale_x[m]) / Q;
+        for (int64_t n = 0; n < N; ++n) out[m * N + n] = (float)acc[m * N + n] * f;
+    }
+    return ORACLE_OK;
+}

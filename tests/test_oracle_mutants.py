@@ -1,0 +1,51 @@
+"""Pin strength: plant one plausible mistake at a time in a copy of the oracle's C
+source, build it, and check that the pin suite (tests/test_oracle_pins.py) fails.
+
+Each mutant is a dropped term, a wrong sign, index or constant, or a wrong
+rounding rule -- the kinds of slip that would otherwise let the oracle agree with
+a CUDA kernel carrying the same slip.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from oracle import build as obuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "fwht_no_stage_scale": ("row[j] = (u + v) * c;", "row[j] = (u + v);"),
+    "fwht_wrong_sign": ("row[j + h] = (u - v) * c;", "row[j + h] = (v - u) * c;"),
+    "fwht_skips_first_stage": ("for (int64_t h = 1; h < K; h *= 2) {", "for (int64_t h = 2; h < K; h *= 2) {"),
+    "rmsnorm_sum_not_mean": ("float mean = ss / (float)K;", "float mean = ss;"),
+    "rmsnorm_no_gain": ("yr[k] = g ? v * g[k] : v;", "yr[k] = v;"),
+    "int8_q_is_128": ("static float q_int8(void) { return 127.0f; }", "static float q_int8(void) { return 128.0f; }"),
+    "int4_sum_not_mean": ("float beta = sum / (float)K;", "float beta = sum;"),
+    "int4_q_is_8": ("return (float)sqrt(7.0); }", "return 8.0f; }"),
+    "round_half_away": ("static float rne(float v) { return nearbyintf(v); }",
+                        "static float rne(float v) { return roundf(v); }"),
+    "int4_clip_low": ("lo = -8.0f;", "lo = -7.0f;"),
+    "pack_wrong_bit_index": ("packed[n * row_bytes + 4 * w + b] |= (uint8_t)(code << (2 * j));",
+                             "packed[n * row_bytes + 4 * w + j] |= (uint8_t)(code << (2 * b));"),
+    "gemm_packed_no_offset": ("s += (int32_t)q[m * K + k] * (int32_t)(code - 1);",
+                              "s += (int32_t)q[m * K + k] * (int32_t)(code);"),
+    "alpha_sum_not_mean": ("return (float)(sum / (double)count);", "return (float)(sum);"),
+    "dequant_times_q": ("float f = (alpha * scale_x[m]) / Q;", "float f = (alpha * scale_x[m]) * Q;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(obuild.SRC).read()
+    assert src.count(before) == 1, f"mutation site for {name} not unique/absent"
+    mut_src = tmp_path / "mutant.c"
+    mut_src.write_text(src.replace(before, after))
+    lib = obuild.build(force=True, src=str(mut_src), out=str(tmp_path / "libmutant.so"))
+    env = dict(os.environ, ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "not slow",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"

@@ -1,0 +1,278 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix,
+never against a retyped copy of the oracle's own formulas.
+
+  * FWHT: the closed-form Sylvester entries (-1)^popcount(i&j)/sqrt(n), scipy's
+    Sylvester Hadamard matrix, H = H^T, H.H = I, H e0 and H 1, Parseval.
+  * RMSNorm: constant rows (closed form), gain linearity, scale invariance.
+  * Activation quantisation: round-half-even/clip tie tables with exact
+    multipliers, the int8 max-code invariant, the int4 code histogram of a
+    normal row against its closed-form probabilities.
+  * Weights: codes in {-1,0,1}; alpha against numpy's float64 mean; the zero
+    fraction of Gaussian weights against 2*Phi(sqrt(2/pi)/2) - 1.
+  * Packing: hand-worked byte layouts, round trip.
+  * GEMM: numpy int64 matmul.
+  * Whole path: the hand-worked tiny cases.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from oracle import ref
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _popcount(v):
+    return bin(v).count("1")
+
+
+# ----------------------------------------------------------------------------- FWHT
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64])
+def test_fwht_matches_closed_form_sylvester(n):
+    H = ref.fwht(np.eye(n, dtype=np.float32))  # row j = H e_j = column j of H
+    closed = np.array([[(-1.0) ** _popcount(i & j) for j in range(n)] for i in range(n)]) / math.sqrt(n)
+    np.testing.assert_allclose(H, closed, rtol=0, atol=4e-7 * max(1, math.log2(n)))
+    sy = scipy.linalg.hadamard(n).astype(np.float64) / math.sqrt(n)
+    np.testing.assert_allclose(H, sy, rtol=0, atol=4e-7 * max(1, math.log2(n)))
+
+
+@pytest.mark.parametrize("n", [2, 8, 64])
+def test_fwht_symmetric_and_involutive(n):
+    H = ref.fwht(np.eye(n, dtype=np.float32)).astype(np.float64)
+    np.testing.assert_allclose(H, H.T, atol=1e-7)
+    HH = ref.fwht(ref.fwht(np.eye(n, dtype=np.float32))).astype(np.float64)
+    np.testing.assert_allclose(HH, np.eye(n), atol=2e-6)
+    np.testing.assert_allclose(H @ H, np.eye(n), atol=2e-6)
+
+
+@pytest.mark.parametrize("n", [256, 4096, 16384])
+def test_fwht_basis_and_parseval(n):
+    e0 = np.zeros((1, n), np.float32)
+    e0[0, 0] = 1
+    np.testing.assert_allclose(ref.fwht(e0)[0], np.full(n, 1 / math.sqrt(n)), rtol=2e-6)
+    ones = np.ones((1, n), np.float32)
+    out = ref.fwht(ones)[0]
+    assert abs(out[0] - math.sqrt(n)) < 1e-5 * math.sqrt(n)
+    assert np.all(out[1:] == 0)
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((3, n)).astype(np.float32)
+    y = ref.fwht(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-5)
+
+
+def test_fwht_against_scipy_matrix_large():
+    n = 2048
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((4, n)).astype(np.float32)
+    H = scipy.linalg.hadamard(n).astype(np.float64) / math.sqrt(n)
+    exact = x.astype(np.float64) @ H.T
+    got = ref.fwht(x).astype(np.float64)
+    np.testing.assert_allclose(got, exact, rtol=0, atol=2e-5)
+
+
+def test_fwht_rejects_non_power_of_two():
+    with pytest.raises(ref.OracleError) as e:
+        ref.fwht(np.ones((1, 6), np.float32))
+    assert e.value.rc == 3
+    with pytest.raises(ref.OracleError):
+        ref.fwht(np.ones((1, 2560), np.float32))
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+def test_rmsnorm_constant_row_closed_form():
+    for c in (1.0, 3.0, 0.001, 250.0):
+        x = np.full((1, 64), c, np.float32)
+        y = ref.rmsnorm(x, eps=1e-5)[0].astype(np.float64)
+        want = c / math.sqrt(c * c + 1e-5)
+        np.testing.assert_allclose(y, want, rtol=3e-7)
+
+
+def test_rmsnorm_zero_row_is_zero():
+    y = ref.rmsnorm(np.zeros((2, 128), np.float32), eps=1e-5)
+    assert np.all(y == 0)
+
+
+def test_rmsnorm_unit_mean_square_and_scale_invariance():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((4, 2560)) * 7).astype(np.float32)
+    y = ref.rmsnorm(x, eps=0.0).astype(np.float64)
+    np.testing.assert_allclose((y * y).mean(axis=1), 1.0, rtol=2e-5)
+    y2 = ref.rmsnorm(x * np.float32(4.0), eps=0.0)
+    np.testing.assert_array_equal(y2, ref.rmsnorm(x, eps=0.0))  # power-of-two scale is exact
+
+
+def test_rmsnorm_gain_is_elementwise():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((3, 256)).astype(np.float32)
+    g = rng.uniform(0.5, 2.0, 256).astype(np.float32)
+    np.testing.assert_array_equal(ref.rmsnorm(x, g), ref.rmsnorm(x) * g)
+
+
+# ----------------------------------------------------------------------------- activation quant
+def test_roundclip_tie_table_int8():
+    d = _gold("roundclip_ties.json")["int8"]
+    y = np.array([d["y"]], np.float32)
+    q, s = ref.act_quant_codes(y, ref.ACT_INT8, eps=d["eps"])
+    assert q[0].tolist() == d["codes"]
+    assert s[0] == np.float32(d["scale"])
+
+
+def test_roundclip_tie_table_int4():
+    d = _gold("roundclip_ties.json")["int4"]
+    y = np.array([d["y"]], np.float32)
+    assert hex(int(y[0, 9].view(np.uint32))) == d["y9_bits"]
+    q, s = ref.act_quant_codes(y, ref.ACT_INT4, eps=d["eps"])
+    assert q[0].tolist() == d["codes"]
+    assert s[0] == np.float32(np.sqrt(7.0)) / np.float32(2.0)
+
+
+def test_int8_max_code_invariant():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((64, 1024)).astype(np.float32)
+    for fw in (False, True):
+        q, s = ref.act_quant(x, fwht_on=fw, mode=ref.ACT_INT8)
+        assert np.all(np.abs(q.astype(np.int32)).max(axis=1) == 127)
+        assert q.min() >= -127  # |y*s| <= 127*gamma/(gamma+eps) < 127.5, so -128 never appears
+
+
+def test_zero_token_gives_zero_codes_and_scale():
+    x = np.zeros((2, 256), np.float32)
+    for mode in (ref.ACT_INT8, ref.ACT_INT4):
+        q, s = ref.act_quant(x, fwht_on=True, mode=mode)
+        assert np.all(q == 0) and np.all(s == 0)
+
+
+def _phi(z):
+    return 0.5 * (1 + math.erf(z / math.sqrt(2)))
+
+
+def test_int4_histogram_matches_normal_closed_form():
+    # RMSNorm'd N(0,1) rows: beta -> E|y| = sqrt(2/pi), step delta = beta/sqrt7; code k has mass
+    # Phi((k+1/2) delta) - Phi((k-1/2) delta), with the tails folded into 7 and -8.
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((64, 16384)).astype(np.float32)
+    q, _ = ref.act_quant(x, mode=ref.ACT_INT4)
+    n = q.size
+    delta = math.sqrt(2 / math.pi) / math.sqrt(7)
+    for k in range(-8, 8):
+        lo = -math.inf if k == -8 else (k - 0.5) * delta
+        hi = math.inf if k == 7 else (k + 0.5) * delta
+        p = (_phi(hi) if hi != math.inf else 1.0) - (_phi(lo) if lo != -math.inf else 0.0)
+        got = np.count_nonzero(q == k) / n
+        sd = math.sqrt(p * (1 - p) / n)
+        assert abs(got - p) < 5 * sd + 1.5e-3 * p, (k, got, p)
+    assert abs(np.count_nonzero(q == 0) / n - 0.1199) < 2e-3
+
+
+def test_shadow_agrees_with_fp32_codes_away_from_ties():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((8, 4096)).astype(np.float32)
+    for mode in (ref.ACT_INT8, ref.ACT_INT4):
+        q, _ = ref.act_quant(x, fwht_on=True, mode=mode)
+        v = ref.shadow(x, fwht_on=True, mode=mode)
+        lo, hi = (-128, 127) if mode == ref.ACT_INT8 else (-8, 7)
+        want = np.clip(np.rint(v), lo, hi)
+        frac = np.abs(v - np.floor(v) - 0.5)
+        far = frac > 1e-3
+        np.testing.assert_array_equal(q[far], want[far])
+
+
+# ----------------------------------------------------------------------------- weights
+def test_ternary_codes_and_alpha():
+    rng = np.random.default_rng(8)
+    W = (rng.standard_normal((300, 512)) * 0.02).astype(np.float32)
+    a = ref.weight_alpha(W)
+    assert a == np.float32(np.mean(np.abs(W.astype(np.float64))))
+    t = ref.ternarize(W, a)
+    assert set(np.unique(t).tolist()) <= {-1, 0, 1}
+
+
+@pytest.mark.slow
+def test_gaussian_weight_zero_fraction_closed_form():
+    # P(t = 0) = P(|w| < (alpha+eps)/2) -> 2*Phi(sqrt(2/pi)/2) - 1 = 0.3101 for Gaussian W.
+    from ternary_weight_bit_b200 import synthetic
+    W = synthetic.decode(1).W.numpy()  # 6912 x 2560 = 17.7 M weights, N(0, 0.02^2)
+    _, _, t = ref.pack_weights(W)
+    p0 = 2 * _phi(0.5 * math.sqrt(2 / math.pi)) - 1
+    assert abs(p0 - 0.3101) < 1e-4
+    f0 = np.count_nonzero(t == 0) / t.size
+    assert abs(f0 - p0) < 1e-3
+    fp = np.count_nonzero(t == 1) / t.size
+    assert abs(fp - (1 - p0) / 2) < 1e-3
+
+
+# ----------------------------------------------------------------------------- packing
+def test_pack_layout_golden():
+    for case in _gold("pack_layout.json")["cases"]:
+        t = np.array([case["t"]], np.int8)
+        p = ref.pack(t)
+        assert p[0].tolist() == case["bytes"], case["derivation"]
+        np.testing.assert_array_equal(ref.unpack(p, 1, t.shape[1]), t)
+
+
+def test_pack_roundtrip_random():
+    rng = np.random.default_rng(9)
+    t = rng.integers(-1, 2, size=(37, 256)).astype(np.int8)
+    p = ref.pack(t)
+    assert p.shape == (37, 64)
+    np.testing.assert_array_equal(ref.unpack(p, 37, 256), t)
+
+
+def test_unpack_flags_invalid_code():
+    p = np.full((1, 4), 0xFF, np.uint8)
+    with pytest.raises(ref.OracleError):
+        ref.unpack(p, 1, 16)
+
+
+# ----------------------------------------------------------------------------- GEMM
+def test_integer_gemm_matches_numpy():
+    rng = np.random.default_rng(10)
+    q = rng.integers(-128, 128, size=(9, 384)).astype(np.int8)
+    t = rng.integers(-1, 2, size=(13, 384)).astype(np.int8)
+    want = q.astype(np.int64) @ t.astype(np.int64).T
+    np.testing.assert_array_equal(ref.gemm_int(q, t), want)
+    np.testing.assert_array_equal(ref.gemm_packed(q, ref.pack(t), 13), want)
+
+
+def test_integer_gemm_extreme_values():
+    K = 16384
+    q = np.full((2, K), -128, np.int8)
+    q[1] = 127
+    t = np.ones((3, K), np.int8)
+    t[1] = -1
+    t[2, ::2] = 0
+    want = q.astype(np.int64) @ t.astype(np.int64).T
+    np.testing.assert_array_equal(ref.gemm_packed(q, ref.pack(t), 3), want)
+
+
+# ----------------------------------------------------------------------------- whole path
+@pytest.mark.parametrize("mode_name", ["int8", "int4"])
+def test_hand_cases(mode_name):
+    g = _gold("hand_cases.json")
+    mode = ref.ACT_INT8 if mode_name == "int8" else ref.ACT_INT4
+    W = np.array(g["W"], np.float32)
+    alpha = ref.weight_alpha(W)
+    assert alpha == np.float32(g["alpha"])
+    t = ref.ternarize(W, alpha, eps=g["eps"])
+    assert t.tolist() == g["t"]
+    for case in g["cases"]:
+        x = np.array([case["x"]], np.float32)
+        y = ref.fwht(ref.rmsnorm(x, eps=g["eps"]))
+        np.testing.assert_allclose(y[0], case["Hy"], rtol=2e-6, atol=1e-6)
+        q, s = ref.act_quant(x, eps=g["eps"], fwht_on=True, mode=mode)
+        acc = ref.gemm_int(q, t)  # K = 4 is below the 16-wide packing granule
+        out = ref.dequant(acc, s, alpha, mode)
+        exp = case[mode_name]
+        assert q[0].tolist() == exp["codes"]
+        np.testing.assert_allclose(s[0], exp["scale"], rtol=2e-6)
+        assert acc[0].tolist() == exp["acc"]
+        np.testing.assert_allclose(out[0], exp["out"], rtol=2e-6, atol=1e-9)
