@@ -229,9 +229,11 @@ int oracle_ternarize(const float *W, int64_t count, float alpha, float eps, int8
  * Step 4b. 2-bit packing of the ternary codes (layout fixed by the library
  * header; restated here from that document, not shared with it).
  * Code map [b158] tl2_lookup_simulation: -1 -> 0, 0 -> 1, +1 -> 2 (3 is never
- * written).  packed is [N][K/4] bytes, row n starting at byte n*K/4.  Inside a row,
- * k = 16*w + 4*j + b (w = k/16, j = (k%16)/4, b = k%4) lives in byte 4*w + b,
- * bits [2j, 2j+2).  K must be a multiple of 16.
+ * written).  packed is [N][K/4] bytes, row n starting at byte n*K/4.  A row is a
+ * sequence of little-endian 32-bit words; word w holds k in [16w, 16w+16): the code
+ * of k = 16*w + 8*h + i (h in {0,1}, i in [0,8)) sits at bits [4i + 2h, 4i + 2h + 2)
+ * of the word, i.e. in byte 4*w + i/2 at bit 4*(i%2) + 2*h.  K must be a multiple
+ * of 16.
  * ------------------------------------------------------------------------- */
 int oracle_pack(const int8_t *t, int64_t N, int64_t K, uint8_t *packed)
 {
@@ -243,8 +245,8 @@ int oracle_pack(const int8_t *t, int64_t N, int64_t K, uint8_t *packed)
             int v = t[n * K + k];
             if (v < -1 || v > 1) return ORACLE_BAD_ARG;
             unsigned code = (unsigned)(v + 1);
-            int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
-            packed[n * row_bytes + 4 * w + b] |= (uint8_t)(code << (2 * j));
+            int64_t w = k / 16, h = (k % 16) / 8, i = k % 8;
+            packed[n * row_bytes + 4 * w + i / 2] |= (uint8_t)(code << (4 * (i % 2) + 2 * h));
         }
     }
     return ORACLE_OK;
@@ -257,8 +259,8 @@ int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *t)
     int bad = 0;
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
-            int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
-            unsigned code = (packed[n * row_bytes + 4 * w + b] >> (2 * j)) & 3u;
+            int64_t w = k / 16, h = (k % 16) / 8, i = k % 8;
+            unsigned code = (packed[n * row_bytes + 4 * w + i / 2] >> (4 * (i % 2) + 2 * h)) & 3u;
             if (code == 3u) bad = 1;
             t[n * K + k] = (int8_t)((int)code - 1);
         }
@@ -294,8 +296,8 @@ int oracle_gemm_packed(const int8_t *q, const uint8_t *packed, int64_t M, int64_
         for (int64_t n = 0; n < N; ++n) {
             int32_t s = 0;
             for (int64_t k = 0; k < K; ++k) {
-                int64_t w = k / 16, j = (k % 16) / 4, b = k % 4;
-                int code = (packed[n * row_bytes + 4 * w + b] >> (2 * j)) & 3;
+                int64_t w = k / 16, h = (k % 16) / 8, i = k % 8;
+                int code = (packed[n * row_bytes + 4 * w + i / 2] >> (4 * (i % 2) + 2 * h)) & 3;
                 s += (int32_t)q[m * K + k] * (int32_t)(code - 1);
             }
             acc[m * N + n] = s;

@@ -27,8 +27,8 @@ MUTANTS = {
     "round_half_away": ("static float rne(float v) { return nearbyintf(v); }",
                         "static float rne(float v) { return roundf(v); }"),
     "int4_clip_low": ("lo = -8.0f;", "lo = -7.0f;"),
-    "pack_wrong_bit_index": ("packed[n * row_bytes + 4 * w + b] |= (uint8_t)(code << (2 * j));",
-                             "packed[n * row_bytes + 4 * w + j] |= (uint8_t)(code << (2 * b));"),
+    "pack_wrong_bit_index": ("packed[n * row_bytes + 4 * w + i / 2] |= (uint8_t)(code << (4 * (i % 2) + 2 * h));",
+                             "packed[n * row_bytes + 4 * w + i / 2] |= (uint8_t)(code << (2 * (i % 2) + 4 * h));"),
     "gemm_packed_no_offset": ("s += (int32_t)q[m * K + k] * (int32_t)(code - 1);",
                               "s += (int32_t)q[m * K + k] * (int32_t)(code);"),
     "alpha_sum_not_mean": ("return (float)(sum / (double)count);", "return (float)(sum);"),
