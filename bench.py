@@ -1,0 +1,522 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 H-BitLinear forward path (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload decode|...]
+
+A step is one pass of the whole per-token path -- RMSNorm, optional FWHT,
+activation quantisation, ternary GEMM/GEMV, fp32 epilogue -- over one batch of
+the workload (weights are packed once, before timing, as a deployment would).
+The default workload is the decode GEMV configuration: int8 absmax, no FWHT,
+M in {1, 4, 8} tokens against W [6912 x 2560] and the transposed W [2560 x 6912];
+one step runs the six forwards.  Inputs are seeded synthetic tensors.
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
+bracketed by a barrier and a device synchronisation, timed with CUDA events on the
+launching stream; the maximum over ranks is reported.  The packed weights rotate
+over enough copies that every step reads them from HBM (total > 4x L2).
+With N > 1 (torchrun), every rank runs its own replica of the workload (the path
+has no cross-GPU exchange); value = tokens of all ranks / max rank time.
+
+--impl reference times the CPU oracle (single-threaded C, test infrastructure)
+on the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary GEMM TOPS & weight GB/s vs roofline; H-BitLinear tokens/s (1 B200)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- workloads
+def workload_cases(name: str):
+    """(label, M, N, K, mode, fwht, x_kind, x_dtype, outliers) of one step of each workload."""
+    if name == "decode":
+        return [("decode", M, N, K, "int8", False, "normal", "f32", 0)
+                for (N, K) in ((6912, 2560), (2560, 6912)) for M in (1, 4, 8)]
+    if name == "prefill":
+        cases = []
+        for w, N, fw in (("Wq", 4096, False), ("Wk", 4096, False), ("Wv", 4096, False), ("Wo", 4096, True),
+                         ("Wup", 11008, False), ("Wgate", 11008, False)):
+            cases.append((w, 4096, N, 4096, "int8", fw, "normal", "bf16", 0))
+        return cases
+    if name == "wdown":
+        return [("wdown", 2048, 2048, 8192, "int4", True, "student_t3", "f32", 82)]
+    m = re.fullmatch(r"msweep_M(\d+)", name)
+    if m:
+        M = int(m.group(1))
+        return [("Wo", M, 4096, 4096, "int4", True, "student_t3", "f32", 41),
+                ("Wdown", M, 4096, 16384, "int4", True, "student_t3", "f32", 164)]
+    raise SystemExit(f"unknown workload {name!r}")
+
+
+WORKLOAD_TEXT = {
+    "decode": "decode GEMV, int8 absmax, no FWHT: X fp32 [M,K] N(0,1), M in {1,4,8}, against ternary W "
+              "[6912x2560] and [2560x6912] (N(0,0.02) absmean-ternarised, 2-bit packed); 6 forwards per step",
+    "prefill": "prefill int8, 7B-like projections: X bf16 [4096,4096]; W Wq/Wk/Wv/Wo [4096x4096] (FWHT on Wo only) "
+               "and Wup/Wgate [11008x4096]; 6 forwards per step",
+    "wdown": "Wdown-style H-BitLinear, int4 absmean + FWHT: X Student-t(3) [2048,8192] with 1% channels x50; "
+             "W [2048x8192]",
+}
+
+
+def workload_text(name):
+    if name in WORKLOAD_TEXT:
+        return WORKLOAD_TEXT[name]
+    return f"M-sweep point ({name}): int4 + FWHT, Student-t(3) X with 1% outlier channels x50; Wo [4096x4096] " \
+           f"and Wdown [4096x16384]"
+
+
+def make_inputs(cases, seed=0):
+    """Host tensors (X, W) for every case, drawn from the shared synthetic generators."""
+    from ternary_weight_bit_b200 import synthetic
+    out = []
+    for i, (label, M, N, K, mode, fwht, xk, xdt, outl) in enumerate(cases):
+        c = synthetic.make_case(label, M, K, N, x_kind=xk, outliers=outl, outlier_gain=50.0 if outl else 20.0,
+                                x_dtype=xdt, fwht=fwht, mode=mode, seed=seed + i)
+        out.append(c)
+    return out
+
+
+def algorithmic_bytes(M, N, K, xdt):
+    """Bytes the method must move per forward: X in, codes/scales round trip, packed W, fp32 out."""
+    xb = 2 if xdt == "bf16" else 4
+    act = M * K * xb + M * K + 4 * M            # act_quant: read X, write codes + scale
+    gemm = N * K // 4 + M * K + 4 * M + 4 * M * N + 4  # packed W, codes, scales, out, alpha
+    return act, gemm
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profile_traffic(kernel_key: str, source_file: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel is unchanged since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_key}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m1 = re.search(r"traffic_bytes_per_launch\s*=\s*([0-9.eE+]+)", text)
+    m2 = re.search(r"source_sha256\s*=\s*([0-9a-f]{64})", text)
+    if not (m1 and m2):
+        return None
+    src = open(os.path.join(ROOT, "ternary_weight_bit_b200", "csrc", source_file), "rb").read()
+    if hashlib.sha256(src).hexdigest() != m2.group(1):
+        return None
+    return float(m1.group(1))
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the GPU works."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1] or [p for (_, p) in self.samples]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in inside if num(p[0]) is not None]
+        mx = [num(p[1]) for p in inside if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(want_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def aggregate(elapsed_ms: float, tokens: float, world: int, backend_device=None):
+    """Max of the per-rank times and sum of the per-rank tokens (rank 0's view)."""
+    if world == 1:
+        return elapsed_ms, tokens
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=backend_device)
+    n = torch.tensor([tokens], dtype=torch.float64, device=backend_device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(cases, budget_s: float, steps: int | None = None):
+    """Time the oracle on a bounded sample of the workload.  Each case runs the full
+    per-token act_quant and the integer GEMM on a sample of output columns; the
+    time is extrapolated to all N columns.  Returns (tokens/s, description, steps)."""
+    import numpy as np
+    from oracle import ref
+    totals = []
+    done = 0
+    t_begin = time.perf_counter()
+    host = make_inputs(cases)
+    packs = []
+    for c in host:
+        packed, alpha, _ = ref.pack_weights(c.W.numpy(), eps=c.eps)
+        packs.append((packed, alpha))
+    # columns per case so one step costs about budget_s / max(steps, 4) seconds
+    target_step = budget_s / max(4, steps or 4)
+    macs = sum(c.M * c.N * c.K for c in host)
+    mac_rate = 2.5e8  # rough single-core rate of the packed-weight loop, refined after the first step
+    frac = min(1.0, target_step * mac_rate / max(macs, 1))
+    while True:
+        t_step = 0.0
+        for c, (packed, alpha) in zip(host, packs):
+            mode = ref.ACT_INT8 if c.mode == "int8" else ref.ACT_INT4
+            ncols = max(1, min(c.N, int(math.ceil(c.N * frac))))
+            X = c.X.float().numpy()
+            t0 = time.perf_counter()
+            q, s = ref.act_quant(X, None, c.eps, c.fwht, mode)
+            t1 = time.perf_counter()
+            acc = ref.gemm_packed(q, packed[:ncols], ncols)
+            ref.dequant(acc, s, alpha, mode)
+            t2 = time.perf_counter()
+            t_step += (t1 - t0) + (t2 - t1) * (c.N / ncols)
+        totals.append(t_step)
+        done += 1
+        elapsed = time.perf_counter() - t_begin
+        if steps is not None and done >= steps:
+            break
+        if steps is None and (elapsed >= budget_s or done >= 50):
+            break
+    tokens = sum(c.M for c in host)
+    per_step = statistics.median(totals)
+    desc = (f"oracle (single-threaded C) on the same inputs: full act_quant per token, integer GEMM on "
+            f"{frac:.2%} of the output columns extrapolated to all N; {done} step(s), median")
+    return tokens / per_step, desc, done, per_step
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import ternary_weight_bit_b200 as tb
+
+    world, rank, local = dist_setup(args.gpus)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    cases = workload_cases(args.workload)
+    host = make_inputs(cases)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+
+    # pack once per weight matrix (offline step, not timed)
+    base = []
+    for c in host:
+        W = c.W.to(dev)
+        packed, alpha = tb.bitnet_pack_ternary(W, eps=c.eps)
+        del W
+        base.append((packed, alpha))
+    packed_bytes = sum(p.numel() for p, _ in base)
+    step_bytes = packed_bytes + sum(c.X.numel() * c.X.element_size() for c in host)
+    R = max(1, min(64, math.ceil(4 * l2 / step_bytes))) if step_bytes < 4 * l2 else 1
+    rot = []  # R copies of (X, packed, alpha, out, ws) per case
+    for r in range(R):
+        items = []
+        for c, (p, a) in zip(host, base):
+            X = c.X.to(dev)
+            ws = torch.empty((max(tb.bitnet_forward_workspace_bytes(c.M, c.K), 256),), dtype=torch.uint8,
+                             device=dev)
+            out = torch.empty((c.M, c.N), dtype=torch.float32, device=dev)
+            items.append((X, p.clone() if r else p, a, out, ws))
+        rot.append(items)
+    torch.cuda.synchronize()
+
+    def step(r):
+        for c, (X, p, a, out, ws) in zip(host, rot[r]):
+            tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for i in range(max(1, min(args.warmup, R))):
+            step(i % R)  # eager warm-up also primes the per-device attribute caches
+    stream.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+    stream.synchronize()
+    assert tb.bitnet_get_last_device_status(stream) == 0
+
+    gpu_uuid = ""
+    try:
+        gpu_uuid = "GPU-" + str(props.uuid) if not str(props.uuid).startswith("GPU-") else str(props.uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    sampler.start()
+    time.sleep(0.3)
+
+    # ------------------------------------------------------------------ timed region
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            graphs[i % R].replay()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    elapsed = e0.elapsed_time(e1)
+    tokens_rank = args.steps * sum(c.M for c in host)
+    max_ms, tokens_all = aggregate(elapsed, tokens_rank, world, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    status = tb.bitnet_get_last_device_status(stream)
+
+    # ------------------------------------------------------------------ dominant kernel alone
+    codes_scales = []
+    for c, (X, p, a, out, ws) in zip(host, rot[0]):
+        codes, scale = tb.bitnet_act_quant(X, eps=c.eps, fwht=c.fwht, mode=c.mode)
+        codes_scales.append((codes, scale))
+    torch.cuda.synchronize(dev)
+
+    def gemm_pass(r):
+        for c, (codes, scale), (X, p, a, out, ws) in zip(host, codes_scales, rot[r]):
+            tb.bitnet_ternary_gemm(codes, scale, c.mode, p, a, c.N, out=out)
+
+    gg = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        gemm_pass(0)
+    stream.synchronize()
+    with torch.cuda.graph(gg, stream=stream):
+        for r in range(R):
+            gemm_pass(r)
+    reps = max(3, min(200, int(2000 / max(1, R * len(host)))))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gg.replay()
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            gg.replay()
+    k1.record(stream)
+    k1.synchronize()
+    gemm_ms = k0.elapsed_time(k1)
+    launches = reps * R * len(host)
+    gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32")[1] for c in host)
+    gemm_ops = reps * R * sum(2.0 * c.M * c.N * c.K for c in host)
+    weight_bytes = reps * R * sum(c.N * c.K / 4 for c in host)
+    avg_launch_s = gemm_ms / 1e3 / launches
+    peaks, peak_src = load_peaks()
+    decode_like = max(c.M for c in host) <= 16
+    if decode_like:
+        achieved = gemm_bytes / launches / avg_launch_s / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": profile_traffic("gemv_decode_traffic", "gemv.cu"),
+                "kernel": "gemv_kernel (mma.sync s8, cluster split-K, TMA ring)",
+                "peak_source": f"hbm_gbs of {peak_src} MEASURED_PEAKS.json (copy, burst)",
+                "avg_launch_us": round(avg_launch_s * 1e6, 3),
+                "bytes_per_launch": round(gemm_bytes / launches)}
+    else:
+        achieved = gemm_ops / launches / avg_launch_s / 1e12
+        bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak = 2.0 * bf16
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": profile_traffic("gemm_tc_traffic", "gemm_sm100.cu"),
+                "kernel": "gemm_tc_kernel (tcgen05 kind::i8, TMEM accumulator)",
+                "peak_source": f"int8 dense = 2 x bf16_tflops of {peak_src} MEASURED_PEAKS.json (nominal ratio)",
+                "avg_launch_us": round(avg_launch_s * 1e6, 3),
+                "ops_per_launch": round(gemm_ops / launches)}
+
+    # ------------------------------------------------------------------ end to end through the public API
+    pinned_x = [c.X.pin_memory() for c in host]
+    pinned_o = [torch.empty((c.M, c.N), dtype=torch.float32).pin_memory() for c in host]
+    e2e_steps = max(3, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for c, hx, ho, (X, p, a, out, ws) in zip(host, pinned_x, pinned_o, rot[0]):
+                X.copy_(hx, non_blocking=True)
+                tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+                ho.copy_(out, non_blocking=True)
+    stream.synchronize()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps):
+            for c, hx, ho, (X, p, a, out, ws) in zip(host, pinned_x, pinned_o, rot[i % R]):
+                X.copy_(hx, non_blocking=True)
+                tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+                ho.copy_(out, non_blocking=True)
+    x1.record(stream)
+    x1.synchronize()
+    e2e_ms = x0.elapsed_time(x1)
+    e2e_max, e2e_tokens = aggregate(e2e_ms, e2e_steps * sum(c.M for c in host), world, dev)
+    h2d = sum(c.X.numel() * c.X.element_size() for c in host)
+    d2h = sum(4 * c.M * c.N for c in host)
+
+    result = None
+    if rank == 0:
+        value = tokens_all / (max_ms / 1e3)
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": workload_text(args.workload), "name": args.workload,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs rotate over {R} copies ({R * step_bytes / 2**20:.0f} MiB > 4x L2)"
+                       if R > 1 else "per-step working set larger than 4x L2",
+                       "cuda_graphs": True, "pdl": True},
+            "roofline": roof,
+            "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
+            "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
+            "e2e": {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "eager calls of bitnet_hbitlinear_forward with pinned host X in and out per step"},
+            "gpu_launches": args.steps * 2 * len(host),
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "device_status": status,
+        }
+    # every rank has finished its GPU work; rank 0 now times the oracle on the host (N=1 only)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        for g in graphs:
+            del g
+        graphs.clear()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, desc, n, per_step = time_oracle(cases, budget_s=args.cpu_budget)
+            result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                      "sample": desc}
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    cases = workload_cases(args.workload)
+    budget = max(10.0, min(150.0, 6.0 * (args.steps + args.warmup)))
+    # warm-up steps are untimed samples too; time exactly --steps steps
+    if args.warmup:
+        time_oracle(cases, budget_s=budget, steps=1)
+    v, desc, n, per_step = time_oracle(cases, budget_s=budget, steps=args.steps)
+    tokens = sum(c[1] for c in cases)
+    result = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": workload_text(args.workload), "name": args.workload},
+        "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": f"{tokens} tokens per step",
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode",
+                    help="decode (default) | prefill | wdown | msweep_M<M>")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * bitnet.h -- C ABI of libbitnet.so, the B200 (sm_100a) H-BitLinear forward path.
+ *
+ * The path (BitNet v2 "H-BitLinear", bitnet_v2_engine.py page, Eq. 1-7):
+ *   1. per-token RMSNorm,
+ *   2. optional Fast Walsh-Hadamard transform along the hidden dimension
+ *      (Eq. 3/4, H_m = (1/sqrt2)[[H,H],[H,-H]], natural order),
+ *   3. per-token activation quantisation, int8 absmax (Eq. 5) or int4 absmean (Eq. 6),
+ *   4. an integer GEMM of those codes against absmean-ternarised weights
+ *      (Eq. 1/2) stored at 2 bits per weight,
+ *   5. an fp32 dequant epilogue, out = acc * alpha * scale_x / Q.
+ *
+ * Conventions for every entry point
+ *   - Shapes: activations X [M][K], weights W [N][K] (the [out][in] layout of
+ *     F.linear), output [M][N]; all row-major and densely packed.
+ *   - Pointers: unless stated otherwise every pointer is a DEVICE pointer owned by
+ *     the caller.  The library never allocates, frees or retains memory; it keeps
+ *     only a per-device cache of kernel attributes and one 4-byte device status word.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on that stream and returns without
+ *     synchronising; results are ready when the stream reaches them.
+ *   - Errors: every call validates its arguments on the host before launching
+ *     anything and returns a bitnet_status_t; nothing throws or aborts.  A kernel
+ *     that gives up on a bounded wait records BITNET_ERR_TIMEOUT in the device
+ *     status word, which bitnet_get_last_device_status() reads.
+ *   - Alignment: every device pointer must be 16-byte aligned (256-byte for
+ *     workspaces).  K must be a multiple of 128 and at most 32768; with the FWHT on
+ *     K must also be a power of two.  M >= 0 and N >= 1; M == 0 is a no-op.
+ *   - eps is the stabiliser of RMSNorm, of the activation scale and of the weight
+ *     scale; the benchmarks use 1e-5.
+ */
+#ifndef BITNET_H
+#define BITNET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BITNET_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,       /* null or misaligned pointer, bad enum, negative size */
+    BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of 128, K > 32768, or similar */
+    BITNET_ERR_NOT_POW2 = 3,          /* FWHT requested with K not a power of two */
+    BITNET_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    BITNET_ERR_TIMEOUT = 5,           /* a kernel gave up on a bounded wait */
+    BITNET_ERR_WORKSPACE = 6          /* workspace missing or smaller than required */
+} bitnet_status_t;
+
+typedef enum {
+    BITNET_ACT_INT8_ABSMAX = 0,  /* Eq. 5: gamma = max|x|, Q = 127, codes in [-128, 127] */
+    BITNET_ACT_INT4_ABSMEAN = 1  /* Eq. 6: beta = mean|x|, Q = sqrt(7), codes in [-8, 7] */
+} bitnet_act_mode_t;
+
+typedef enum {
+    BITNET_F32 = 0,
+    BITNET_BF16 = 1
+} bitnet_dtype_t;
+
+/*
+ * Packed ternary weight layout (this library's format).
+ *   Codes: t in {-1, 0, +1} is stored as t + 1 in {0, 1, 2} (the map of the
+ *   tl2_lookup_simulation listing in the youngju.dev BitNet transcription); the
+ *   value 3 is never written and its meaning is unspecified.
+ *   packed is [N][K/4] bytes; row n starts at byte n*K/4.  A row is a sequence of
+ *   little-endian 32-bit words; word w holds k in [16w, 16w+16): the code of
+ *   k = 16w + 8h + i (h in {0,1}, i in [0,8)) occupies bits [4i+2h, 4i+2h+2) of the
+ *   word -- byte 4w + i/2, bit 4(i%2) + 2h.  (One shift and a 0x33333333 mask put
+ *   eight codes in eight nibbles; one byte permute makes four of them signed int8.)
+ */
+
+/* --------------------------------------------------------------------------
+ * bitnet_pack_ternary -- step 4a, once per weight matrix (not on the per-token path).
+ * Definition: bitnet_v2_engine.py page, Eq. 1/2 and quantize_weight_ternary:
+ *   alpha = mean|W| over all N*K entries (summed in double, one rounding to float),
+ *   t = RoundClip(W / (alpha + eps), -1, 1) in fp32, rounding half to even.
+ *   W       [N][K] fp32, device, read only.
+ *   packed  [N][K/4] bytes, device, written (layout above).
+ *   alpha   one fp32, device, written: the per-tensor weight scale used by the GEMM.
+ *   ws      device scratch of at least bitnet_pack_workspace_bytes() bytes.
+ * Deterministic: the same W always gives the same bytes and alpha.
+ * ------------------------------------------------------------------------ */
+BITNET_API size_t bitnet_pack_workspace_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status_t bitnet_pack_ternary(const float *W, int64_t N, int64_t K, float eps,
+                                    uint8_t *packed, float *alpha,
+                                    void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * bitnet_act_quant -- steps 1-3 fused, one HBM pass per token.
+ * Definition: bitnet_v2_engine.py page, HBitLinear.forward (RMSNorm -> Hadamard ->
+ * quantise), fast_hadamard_transform (Eq. 3/4), quantize_act_int8 (Eq. 5),
+ * quantize_act_int4 (Eq. 6):
+ *   r = 1/sqrt(mean(x^2) + eps);  y = (x*r)*gain;  if fwht: y = H_K y;
+ *   int8: gamma = max|y|, s = 127/(gamma+eps), code = clamp(rne(y*s), -128, 127);
+ *   int4: beta = mean|y|, s = sqrt7/(beta+eps), code = clamp(rne(y*s), -8, 7).
+ *   X        [M][K], fp32 or bf16 (xdt), device, read only.
+ *   gain     [K] fp32 RMSNorm gain, device; NULL means all ones.
+ *   fwht     0 = off, 1 = on (K must then be a power of two: BITNET_ERR_NOT_POW2).
+ *   codes    [M][K] int8, device, written (int4 codes are stored one per byte).
+ *   scale_x  [M] fp32, device, written: gamma (int8) or beta (int4), without eps.
+ * The GPU sums and rotates in a different order than a sequential reference;
+ * a code may then differ by one where y*s lies within rounding of a half-integer.
+ * ------------------------------------------------------------------------ */
+BITNET_API bitnet_status_t bitnet_act_quant(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                 const float *gain, float eps, int fwht,
+                                 bitnet_act_mode_t mode, int8_t *codes, float *scale_x,
+                                 void *stream);
+
+/* --------------------------------------------------------------------------
+ * bitnet_ternary_gemm -- steps 4b-5: integer GEMM on packed ternary weights plus
+ * the fp32 dequant epilogue.
+ * Definition: bitnet_v2_engine.py page, HBitLinear.forward (F.linear of the
+ * quantised operands); BitLinear_b158.forward in the youngju.dev transcription
+ * (integer product, then output * (w_scale * x_scale) / Q):
+ *   acc[m][n] = sum_k codes[m][k] * t[n][k]           (exact int32)
+ *   out[m][n] = (float)acc[m][n] * ((alpha * scale_x[m]) / Q),  Q = 127 or sqrt7.
+ *   codes    [M][K] int8, device, read only.
+ *   scale_x  [M] fp32, device, read only.
+ *   packed   [N][K/4] bytes (layout above), device, read only.
+ *   alpha    one fp32, device, read only.
+ *   out      [M][N] fp32, device, written.
+ *   acc_out  [M][N] int32, device, written when not NULL (for exactness checks).
+ * M <= 16 runs the weight-streaming decode kernel (tensor-core mma.sync, cluster
+ * split-K); larger M runs the tcgen05 int8 tensor-core GEMM with TMEM accumulators.
+ * ------------------------------------------------------------------------ */
+BITNET_API bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x,
+                                    bitnet_act_mode_t mode, const uint8_t *packed,
+                                    const float *alpha, int64_t M, int64_t N, int64_t K,
+                                    float *out, int32_t *acc_out, void *stream);
+
+/* --------------------------------------------------------------------------
+ * bitnet_hbitlinear_forward -- the whole path: bitnet_act_quant into the
+ * workspace, then bitnet_ternary_gemm from it (the second kernel is launched with
+ * programmatic dependent launch so its weight stream starts while the first runs).
+ * Definition: bitnet_v2_engine.py page, HBitLinear.forward, Eq. 7.
+ *   Arguments as in the two calls above; ws is device scratch of at least
+ *   bitnet_forward_workspace_bytes(M, K) bytes holding the int8 codes and the
+ *   per-token scales between the two kernels (BITNET_ERR_WORKSPACE if smaller).
+ * ------------------------------------------------------------------------ */
+BITNET_API size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K);
+BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M,
+                                          int64_t K, const float *gain, float eps, int fwht,
+                                          bitnet_act_mode_t mode, const uint8_t *packed,
+                                          const float *alpha, int64_t N, float *out,
+                                          void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Status and diagnostics (no counterpart on the pages).
+ * bitnet_status_string: static English text for a status code.
+ * bitnet_get_last_device_status: synchronises `stream`, returns the status word
+ *   the kernels record on a bounded-wait timeout (BITNET_OK if none) and clears it.
+ * bitnet_selftest_wait_timeout: launches one CTA that waits on a barrier nothing
+ *   will ever complete, with the given limit in microseconds (1..1000000); the
+ *   wait gives up, records BITNET_ERR_TIMEOUT and the kernel returns normally.
+ *   Used by the tests to exercise the timeout path without hanging the GPU.
+ * bitnet_abi_version: BITNET_ABI_VERSION of the loaded library.
+ * ------------------------------------------------------------------------ */
+BITNET_API const char *bitnet_status_string(bitnet_status_t status);
+BITNET_API bitnet_status_t bitnet_get_last_device_status(void *stream);
+BITNET_API bitnet_status_t bitnet_selftest_wait_timeout(uint32_t limit_us, void *stream);
+BITNET_API int bitnet_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_H */

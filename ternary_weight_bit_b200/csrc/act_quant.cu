@@ -1,0 +1,398 @@
+// act_quant.cu -- steps 1-3 of the H-BitLinear forward, fused: per-token RMSNorm,
+// optional Fast Walsh-Hadamard transform, int8-absmax / int4-absmean quantisation.
+//
+// Method: bitnet_v2_engine.py page -- HBitLinear.forward (normalise, rotate,
+// quantise), fast_hadamard_transform and Eq. 3/4 (H_m = (1/sqrt2)[[H,H],[H,-H]]),
+// quantize_act_int8 (Eq. 5) and quantize_act_int4 (Eq. 6).
+//
+// One CTA per token; X is read from HBM exactly once (128-bit loads) and the
+// codes are written once.  Everything in between stays on chip.
+//
+// FWHT kernel (K = 2^LOGK): each thread owns E = 2^ELOG elements.  The transform
+// runs as unnormalised radix-2 butterflies (a+b, a-b) over bits 0, 1, ..., LOGK-1
+// in increasing order, in phases of ELOG bits: inside a phase the butterflies are
+// in registers; between phases the token is transposed through shared memory so
+// that the next ELOG index bits become register bits.  The 1/sqrt2 per stage is
+// folded into one multiplier 2^(-LOGK/2) applied together with the RMSNorm factor
+// (exact for even LOGK).  This reorders the roundings of the page's per-stage
+// scaling; results differ from it only in the last bits.
+#include "common.cuh"
+
+namespace bitnet {
+
+namespace {
+
+// ------------------------------------------------------------------ reductions
+template <int T>
+__device__ __forceinline__ float block_sum(float v, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    constexpr int W = T / 32;
+    if constexpr (W == 1) {
+        return v;
+    } else {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        __syncthreads();  // red may still be read from a previous reduction
+        if (lane == 0) red[warp] = v;
+        __syncthreads();
+        float s = lane < W ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        return s;
+    }
+}
+
+template <int T>
+__device__ __forceinline__ float block_max(float v, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    constexpr int W = T / 32;
+    if constexpr (W == 1) {
+        return v;
+    } else {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        __syncthreads();
+        if (lane == 0) red[warp] = v;
+        __syncthreads();
+        float s = lane < W ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, o));
+        return s;
+    }
+}
+
+// ------------------------------------------------------------------ quantiser
+// Round-clip y*s to [lo, hi] with round-half-to-even, returned as the low byte of
+// the result: adding 1.5*2^23 rounds an fp32 in [-2^22, 2^22] to the nearest
+// integer (ties to even) and leaves that integer in the low mantissa bits.
+__device__ __forceinline__ uint32_t quant_byte(float y, float s, float lo, float hi) {
+    const float v = fminf(fmaxf(__fmul_rn(y, s), lo), hi);
+    return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xFFu;
+}
+
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+struct QuantParams {
+    float s, lo, hi;
+};
+
+__device__ __forceinline__ QuantParams quant_params(float stat, float eps, int mode) {
+    QuantParams q;
+    if (mode == BITNET_ACT_INT8_ABSMAX) {
+        q.s = __fdiv_rn(127.0f, __fadd_rn(stat, eps));
+        q.lo = -128.0f;
+        q.hi = 127.0f;
+    } else {
+        q.s = __fdiv_rn(2.64575131106459059f, __fadd_rn(stat, eps));
+        q.lo = -8.0f;
+        q.hi = 7.0f;
+    }
+    return q;
+}
+
+__device__ __forceinline__ float rms_factor(float ss, int K, float eps) {
+    return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+}
+
+// Load 8 consecutive elements (fp32 or bf16) starting at element index `idx`.
+template <bool BF16>
+__device__ __forceinline__ void load8(const void *X, int64_t idx, float *v) {
+    if constexpr (BF16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(X) + idx));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(X) + idx);
+        const float4 a = __ldg(p), b = __ldg(p + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void load4(const void *X, int64_t idx, float *v) {
+    if constexpr (BF16) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(X) + idx));
+        v[0] = __uint_as_float(u.x << 16);
+        v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        v[2] = __uint_as_float(u.y << 16);
+        v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(X) + idx));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    }
+}
+
+// ------------------------------------------------------------------ FWHT kernel
+template <int LOGK>
+struct FwhtShape {
+    static constexpr int K = 1 << LOGK;
+    static constexpr int ELOG = (LOGK - 5) < 5 ? (LOGK - 5) : 5;  // elements per thread = 2^ELOG
+    static constexpr int E = 1 << ELOG;
+    static constexpr int T = K / E;  // threads per CTA (>= 32)
+    static constexpr int PHASES = (LOGK + ELOG - 1) / ELOG;
+};
+
+// Index of register r of thread tid in phase p: the register bits are
+// [lo, lo+nb) plus, in a short last phase, the low `pass` bits as passengers.
+template <int LOGK, int ELOG>
+__device__ __forceinline__ int phase_index(int p, int tid, int r) {
+    const int lo = p * ELOG;
+    const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
+    const int pass = ELOG - nb;
+    const int tl = lo - pass;
+    const int r_pass = r & ((1 << pass) - 1);
+    const int r_hi = r >> pass;
+    return r_pass | ((tid & ((1 << tl) - 1)) << pass) | (r_hi << lo) | ((tid >> tl) << (lo + nb));
+}
+
+// Bank-spreading permutation of the shared-memory copy of a token.
+__device__ __forceinline__ int swz(int i) { return i ^ ((i >> 5) & 31); }
+
+template <int LOGK, bool BF16>
+__global__ void __launch_bounds__(FwhtShape<LOGK>::T)
+act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain, float eps, int mode,
+                      int8_t *__restrict__ codes, float *__restrict__ scale_x) {
+    using S = FwhtShape<LOGK>;
+    constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
+    extern __shared__ __align__(16) float sm[];  // K floats
+    __shared__ float red[32];
+
+    pdl_launch_dependents();  // the GEMM may start streaming weights now
+
+    const int tid = threadIdx.x;
+    const int64_t row = (int64_t)blockIdx.x * K;
+    float v[E];
+
+    // Phase 0 layout: thread tid owns the E contiguous elements [tid*E, tid*E + E).
+    if constexpr (E >= 8) {
+#pragma unroll
+        for (int c = 0; c < E / 8; ++c) load8<BF16>(X, row + tid * E + 8 * c, v + 8 * c);
+    } else {
+        load4<BF16>(X, row + tid * E, v);
+    }
+
+    float ss = 0.0f;
+#pragma unroll
+    for (int r = 0; r < E; ++r) ss = fmaf(v[r], v[r], ss);
+    ss = block_sum<T>(ss, red);
+    const float rn = rms_factor(ss, K, eps);
+
+    if (gain != nullptr) {
+#pragma unroll
+        for (int r = 0; r < E; ++r) v[r] = __fmul_rn(v[r], __ldg(gain + tid * E + r));
+    }
+
+    // Butterflies over all LOGK bits, in increasing bit order.
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        if (p > 0) {
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < E; ++r) sm[swz(phase_index<LOGK, ELOG>(p - 1, tid, r))] = v[r];
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < E; ++r) v[r] = sm[swz(phase_index<LOGK, ELOG>(p, tid, r))];
+        }
+        const int lo = p * ELOG;
+        const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
+        const int pass = ELOG - nb;
+#pragma unroll
+        for (int b = 0; b < ELOG; ++b) {
+            if (b >= pass) {
+                const int h = 1 << b;
+#pragma unroll
+                for (int r = 0; r < E; ++r) {
+                    if ((r & h) == 0) {
+                        const float a = v[r], c = v[r | h];
+                        v[r] = __fadd_rn(a, c);
+                        v[r | h] = __fsub_rn(a, c);
+                    }
+                }
+            }
+        }
+    }
+
+    // y = z * (r * 2^(-LOGK/2))
+    const float p2 = __int_as_float((127 - LOGK / 2) << 23);  // 2^(-floor(LOGK/2)), exact
+    const float hs = (LOGK & 1) ? __fmul_rn(0.70710678118654752f, p2) : p2;
+    const float rho = __fmul_rn(rn, hs);
+    float stat;
+    if (mode == BITNET_ACT_INT8_ABSMAX) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+            v[r] = __fmul_rn(v[r], rho);
+            mx = fmaxf(mx, fabsf(v[r]));
+        }
+        stat = block_max<T>(mx, red);
+    } else {
+        float sa = 0.0f;
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+            v[r] = __fmul_rn(v[r], rho);
+            sa += fabsf(v[r]);
+        }
+        stat = __fdiv_rn(block_sum<T>(sa, red), (float)K);
+    }
+    const QuantParams q = quant_params(stat, eps, mode);
+
+    // Store the codes in the last phase's layout.
+    constexpr int LASTLO = (P - 1) * ELOG;
+    constexpr int LASTNB = (LOGK - LASTLO) < ELOG ? (LOGK - LASTLO) : ELOG;
+    constexpr int LASTPASS = ELOG - LASTNB;
+    int8_t *out = codes + row;
+    if constexpr (LASTPASS >= 2) {
+#pragma unroll
+        for (int r = 0; r < E; r += 4) {
+            const int i = phase_index<LOGK, ELOG>(P - 1, tid, r);
+            const uint32_t w = pack4(quant_byte(v[r], q.s, q.lo, q.hi), quant_byte(v[r + 1], q.s, q.lo, q.hi),
+                                     quant_byte(v[r + 2], q.s, q.lo, q.hi), quant_byte(v[r + 3], q.s, q.lo, q.hi));
+            *reinterpret_cast<uint32_t *>(out + i) = w;
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+            const int i = phase_index<LOGK, ELOG>(P - 1, tid, r);
+            out[i] = (int8_t)quant_byte(v[r], q.s, q.lo, q.hi);
+        }
+    }
+    if (tid == 0) scale_x[blockIdx.x] = stat;
+}
+
+// ------------------------------------------------------------------ plain kernel (no FWHT)
+// Thread tid owns the float4 groups j = it*T + tid, it in [0, NV); K % 4 == 0.
+template <int T, int NV, bool BF16>
+__global__ void __launch_bounds__(T)
+act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gain, int K, float eps,
+                       int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x) {
+    __shared__ float red[32];
+    pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    const int64_t row = (int64_t)blockIdx.x * K;
+    const int K4 = K >> 2;
+    float v[NV][4];
+    float ss = 0.0f;
+#pragma unroll
+    for (int it = 0; it < NV; ++it) {
+        const int j = it * T + tid;
+        if (j < K4) {
+            load4<BF16>(X, row + 4 * j, v[it]);
+        } else {
+            v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss = fmaf(v[it][e], v[it][e], ss);
+    }
+    ss = block_sum<T>(ss, red);
+    const float rn = rms_factor(ss, K, eps);
+
+    float part = 0.0f;
+#pragma unroll
+    for (int it = 0; it < NV; ++it) {
+        const int j = it * T + tid;
+        float g[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+        if (gain != nullptr && j < K4) {
+            const float4 gg = __ldg(reinterpret_cast<const float4 *>(gain) + j);
+            g[0] = gg.x; g[1] = gg.y; g[2] = gg.z; g[3] = gg.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float y = __fmul_rn(v[it][e], rn);
+            if (gain != nullptr) y = __fmul_rn(y, g[e]);
+            v[it][e] = y;
+            part = mode == BITNET_ACT_INT8_ABSMAX ? fmaxf(part, fabsf(y)) : part + fabsf(y);
+        }
+    }
+    float stat;
+    if (mode == BITNET_ACT_INT8_ABSMAX) {
+        stat = block_max<T>(part, red);
+    } else {
+        stat = __fdiv_rn(block_sum<T>(part, red), (float)K);
+    }
+    const QuantParams q = quant_params(stat, eps, mode);
+#pragma unroll
+    for (int it = 0; it < NV; ++it) {
+        const int j = it * T + tid;
+        if (j < K4) {
+            const uint32_t w = pack4(quant_byte(v[it][0], q.s, q.lo, q.hi), quant_byte(v[it][1], q.s, q.lo, q.hi),
+                                     quant_byte(v[it][2], q.s, q.lo, q.hi), quant_byte(v[it][3], q.s, q.lo, q.hi));
+            reinterpret_cast<uint32_t *>(codes + row)[j] = w;
+        }
+    }
+    if (tid == 0) scale_x[blockIdx.x] = stat;
+}
+
+template <int LOGK, bool BF16>
+cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
+                        float *scale_x, cudaStream_t s) {
+    using S = FwhtShape<LOGK>;
+    const size_t smem = (size_t)S::K * sizeof(float);
+    auto kern = act_quant_fwht_kernel<LOGK, BF16>;
+    if (smem > 48 * 1024) {
+        static bool done[kMaxDevices] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev >= kMaxDevices || !done[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            if (dev < kMaxDevices) done[dev] = true;
+        }
+    }
+    kern<<<(unsigned)M, S::T, smem, s>>>(X, gain, eps, mode, codes, scale_x);
+    return cudaGetLastError();
+}
+
+template <int NV, bool BF16>
+cudaError_t launch_plain(const void *X, int64_t M, int K, const float *gain, float eps, int mode,
+                         int8_t *codes, float *scale_x, cudaStream_t s) {
+    constexpr int T = 256;
+    act_quant_plain_kernel<T, NV, BF16><<<(unsigned)M, T, 0, s>>>(X, gain, K, eps, mode, codes, scale_x);
+    return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t dispatch(const void *X, int64_t M, int K, const float *gain, float eps, int fwht, int mode,
+                     int8_t *codes, float *scale_x, cudaStream_t s) {
+    if (fwht) {
+        switch (__builtin_ctz((unsigned)K)) {
+            case 7: return launch_fwht<7, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 8: return launch_fwht<8, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 9: return launch_fwht<9, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 10: return launch_fwht<10, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 11: return launch_fwht<11, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 12: return launch_fwht<12, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 13: return launch_fwht<13, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 14: return launch_fwht<14, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 15: return launch_fwht<15, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    const int nv = (int)ceil_div(K / 4, 256);
+    if (nv <= 1) return launch_plain<1, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 2) return launch_plain<2, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 4) return launch_plain<4, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 8) return launch_plain<8, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 16) return launch_plain<16, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 32) return launch_plain<32, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+// Host entry used by the ABI layer (arguments already validated).
+cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
+                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    return bf16 ? dispatch<true>(X, M, K, gain, eps, fwht, mode, codes, scale_x, s)
+                : dispatch<false>(X, M, K, gain, eps, fwht, mode, codes, scale_x, s);
+}
+
+}  // namespace bitnet

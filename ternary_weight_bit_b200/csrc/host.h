@@ -1,0 +1,42 @@
+// host.h -- host-side declarations shared by the libbitnet translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bitnet {
+
+// Encode a 2-D tiled TMA descriptor over a row-major byte matrix [rows][row_bytes]
+// (element type uint8).  box = {box_x bytes, box_y rows}; swizzle is one of
+// CU_TENSOR_MAP_SWIZZLE_{NONE,32B,64B,128B}.  Out-of-bounds boxes read as zero.
+bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_x, uint32_t box_y, CUtensorMapSwizzle swizzle);
+
+// Per-device address of the library's device status word.
+int *device_status_ptr();
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
+                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s);
+
+size_t pack_workspace_bytes();
+cudaError_t launch_pack(const float *W, int64_t N, int64_t K, float eps, uint8_t *packed, float *alpha,
+                        void *ws, cudaStream_t s);
+
+// Decode path (M <= 16): weight-streaming mma.sync kernel with cluster split-K.
+cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
+                        const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
+                        bool pdl, cudaStream_t s);
+
+// Prefill path: tcgen05 int8 tensor-core GEMM with TMEM accumulators.
+cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
+                           const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
+                           bool pdl, cudaStream_t s);
+
+// Launch the timeout self-test kernel.
+cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);
+
+}  // namespace bitnet

@@ -1,0 +1,73 @@
+"""Comparison rules between the CUDA path and the oracle (shared by the GPU tests,
+the smoke check and the benchmark's parity spot checks).
+
+Rules (from the BitNet v2 page's Eq. 5/6 and the exactness of integer arithmetic):
+  * Packed weight bytes and alpha: identical.
+  * int32 accumulators on the same codes: identical.
+  * fp32 output on the same codes and scales: out = (float)acc * f, f computed in
+    the same IEEE order on both sides, so identical up to the scale's own rounding.
+  * Activation codes: the GPU sums and rotates in another order than the oracle's
+    sequential fp32 loops, so a code may differ by exactly one, only where the exact
+    (fp64) pre-rounding value lies within TIE_TOL of the half-integer between the
+    two codes, and on at most FLIP_RATE of the elements (never fewer than one
+    allowed flip for tiny inputs).
+  * End-to-end output: per token, max|gpu - oracle| <= 1e-3 * max|oracle| plus
+    one weight step (alpha * scale_x / Q) per flipped code of that token.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+TIE_TOL = 2e-3      # code units; fp32 reordering errors are ~1e-5 of a code
+FLIP_RATE = 1e-4    # at most this fraction of codes may differ (by one)
+OUT_RTOL = 1e-3     # max relative error of the fp32 output (normwise per token)
+SQRT7 = np.float32(math.sqrt(7.0))
+
+
+def q_of(mode: int) -> np.float32:
+    return np.float32(127.0) if mode == 0 else SQRT7
+
+
+def check_codes(gpu: np.ndarray, ora: np.ndarray, shadow: np.ndarray, label: str = "") -> int:
+    """Assert the near-tie rule; return the number of flipped codes."""
+    gpu = gpu.astype(np.int32)
+    ora = ora.astype(np.int32)
+    d = gpu - ora
+    flips = np.nonzero(d)
+    nflip = len(flips[0])
+    if nflip:
+        assert np.abs(d).max() == 1, f"{label}: a code differs by {np.abs(d).max()}"
+        boundary = (gpu[flips] + ora[flips]) / 2.0
+        dist = np.abs(shadow[flips] - boundary)
+        worst = float(dist.max())
+        assert worst <= TIE_TOL, f"{label}: a flipped code is {worst:.3g} code units from its rounding tie"
+    allowed = max(1, int(math.floor(FLIP_RATE * gpu.size)))
+    assert nflip <= allowed, f"{label}: {nflip} flipped codes of {gpu.size} (allowed {allowed})"
+    return nflip
+
+
+def check_scale(gpu: np.ndarray, ora: np.ndarray, label: str = "") -> None:
+    np.testing.assert_allclose(gpu, ora, rtol=2e-5, atol=0, err_msg=f"{label}: per-token scale")
+
+
+def check_out_same_codes(gpu_out: np.ndarray, ref_out: np.ndarray, label: str = "") -> None:
+    """Output computed from identical codes: elementwise relative error bound."""
+    denom = np.maximum(np.abs(ref_out), 1e-30)
+    rel = np.abs(gpu_out.astype(np.float64) - ref_out) / denom
+    rel[ref_out == 0] = np.abs(gpu_out[ref_out == 0])
+    assert float(rel.max()) <= 1e-5, f"{label}: max elementwise rel err {float(rel.max()):.3g}"
+
+
+def check_out_end_to_end(gpu_out, ora_out, gpu_codes, ora_codes, ora_scale, alpha, mode, label=""):
+    """Normwise per-token bound, widened by one weight step per flipped code."""
+    flips = (gpu_codes != ora_codes).sum(axis=1)
+    step = np.float64(alpha) * ora_scale.astype(np.float64) / float(q_of(mode))
+    err = np.abs(gpu_out.astype(np.float64) - ora_out).max(axis=1)
+    ref = np.abs(ora_out).max(axis=1)
+    bound = OUT_RTOL * ref + flips * step * 1.001 + 1e-30
+    bad = np.nonzero(err > bound)[0]
+    assert len(bad) == 0, (f"{label}: token {bad[0]} err {err[bad[0]]:.3g} > bound {bound[bad[0]]:.3g} "
+                           f"(flips {flips[bad[0]]})")
+    assert float((err / np.maximum(ref, 1e-30)).max()) <= OUT_RTOL + float((flips * step / np.maximum(ref, 1e-30)).max())

@@ -1,0 +1,89 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, it exports
+every function include/bitnet.h declares, and its argument validation rejects bad
+calls before any CUDA work is attempted."""
+import ctypes
+
+import pytest
+
+from ternary_weight_bit_b200 import _native
+
+
+@pytest.fixture(scope="module")
+def L():
+    return _native.load()
+
+
+def test_header_declares_the_boundary():
+    names = _native.declared_symbols()
+    for required in ("bitnet_pack_ternary", "bitnet_act_quant", "bitnet_ternary_gemm",
+                     "bitnet_hbitlinear_forward"):
+        assert required in names
+    assert len(names) >= 10
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _native.declared_symbols():
+        assert hasattr(L, name), f"{name} declared in bitnet.h but not exported"
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.bitnet_abi_version() == 1
+    for s in range(7):
+        assert L.bitnet_status_string(s)
+    assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
+
+
+def test_workspace_sizes(L):
+    assert L.bitnet_forward_workspace_bytes(0, 256) == 0
+    assert L.bitnet_forward_workspace_bytes(1, 256) == 256 + 256
+    assert L.bitnet_forward_workspace_bytes(3, 2560) == 7680 + 256
+    assert L.bitnet_forward_workspace_bytes(100, 128) == 12800 + 512
+    assert L.bitnet_pack_workspace_bytes(6912, 2560) >= 8 * 1184
+
+
+P = ctypes.c_void_p
+FAKE = P(4096)  # never dereferenced: validation fails first
+
+
+def test_validation_rejects_bad_shapes(L):
+    s = P(0)
+    # K not a multiple of 128
+    assert L.bitnet_act_quant(FAKE, 0, 4, 100, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_UNSUPPORTED_SHAPE
+    # K too large
+    assert L.bitnet_act_quant(FAKE, 0, 4, 65536, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_UNSUPPORTED_SHAPE
+    # FWHT with K not a power of two (the page's ValueError)
+    assert L.bitnet_act_quant(FAKE, 0, 4, 2560, None, 1e-5, 1, 0, FAKE, FAKE, s) == _native.ERR_NOT_POW2
+    assert L.bitnet_hbitlinear_forward(FAKE, 0, 4, 6912, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, FAKE, 1 << 20,
+                                       s) == _native.ERR_NOT_POW2
+    # bad enums
+    assert L.bitnet_act_quant(FAKE, 7, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_act_quant(FAKE, 0, 4, 256, None, 1e-5, 0, 9, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 3, FAKE, FAKE, 4, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+    # negative sizes, N = 0
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, -1, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 0, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+
+
+def test_validation_rejects_bad_pointers(L):
+    s = P(0)
+    assert L.bitnet_act_quant(None, 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_act_quant(P(4100), 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, None, FAKE, 4, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 16, 256, P(4104), None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_pack_ternary(FAKE, 16, 256, 1e-5, FAKE, FAKE, None, 0, s) == _native.ERR_WORKSPACE
+    assert L.bitnet_pack_ternary(FAKE, 16, 256, 1e-5, FAKE, P(4108), FAKE, 1 << 20, s) == _native.ERR_INVALID_ARG
+    # forward workspace too small, or misaligned
+    assert L.bitnet_hbitlinear_forward(FAKE, 0, 4, 256, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, FAKE, 16,
+                                       s) == _native.ERR_WORKSPACE
+    assert L.bitnet_hbitlinear_forward(FAKE, 0, 4, 256, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, P(4096 + 16),
+                                       1 << 20, s) == _native.ERR_WORKSPACE
+    assert L.bitnet_selftest_wait_timeout(0, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_selftest_wait_timeout(2000000, s) == _native.ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_noop(L):
+    s = P(0)
+    assert L.bitnet_act_quant(None, 0, 0, 256, None, 1e-5, 1, 0, None, None, s) == _native.OK
+    assert L.bitnet_ternary_gemm(None, None, 0, None, None, 0, 16, 256, None, None, s) == _native.OK
+    assert L.bitnet_hbitlinear_forward(None, 0, 0, 256, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, None, 0,
+                                       s) == _native.OK

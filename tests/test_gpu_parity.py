@@ -1,0 +1,286 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every comparison follows tests/parity.py: packed bytes, alpha and int32
+accumulators bit-exact; activation codes equal except for one-step flips at
+rounding near-ties; fp32 outputs within the stated relative bounds.  Shapes span
+several tiles plus ragged tails (M, N not multiples of any tile; K with a
+128-wide tail), the degenerate inputs (zero tokens, one token) and the full
+benchmark sizes on sampled tokens.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import parity
+import ternary_weight_bit_b200 as tb
+from oracle import ref
+from ternary_weight_bit_b200 import synthetic
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+MODES = {"int8": ref.ACT_INT8, "int4": ref.ACT_INT4}
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    yield
+    assert tb.bitnet_get_last_device_status() == 0, "a kernel recorded a timeout"
+
+
+def _heavy_x(M, K, seed, outliers=True):
+    g = synthetic.generator(seed)
+    X = synthetic.student_t3((M, K), g)
+    if outliers:
+        X[:, synthetic.outlier_channels(K, max(1, K // 100), g)] *= 50.0
+    return X
+
+
+# ----------------------------------------------------------------------------- pack
+@pytest.mark.parametrize("N,K", [(256, 256), (300, 384), (6912, 2560), (2560, 6912)])
+def test_pack_matches_oracle(N, K):
+    W = synthetic.gaussian((N, K), 0.02, synthetic.generator(N + K))
+    packed, alpha = tb.bitnet_pack_ternary(W.to(DEV), eps=1e-5)
+    p_ref, a_ref, _ = ref.pack_weights(W.numpy(), eps=1e-5)
+    assert host(alpha)[0] == a_ref
+    np.testing.assert_array_equal(host(packed), p_ref)
+
+
+def test_pack_is_deterministic():
+    W = synthetic.gaussian((1024, 1024), 0.02, synthetic.generator(5)).to(DEV)
+    p1, a1 = tb.bitnet_pack_ternary(W)
+    p2, a2 = tb.bitnet_pack_ternary(W)
+    assert torch.equal(p1, p2) and torch.equal(a1, a2)
+
+
+# ----------------------------------------------------------------------------- act_quant
+FWHT_K = [128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768]
+PLAIN_K = [128, 384, 2560, 6912, 16384]
+
+
+def _act_case(M, K, fwht, mode, xdtype, use_gain, seed=0):
+    X = _heavy_x(M, K, seed + K)
+    if xdtype == "bf16":
+        X = X.to(torch.bfloat16)
+    gain = None
+    if use_gain:
+        gain = torch.rand(K, generator=synthetic.generator(seed + 1)) + 0.5
+    Xd = X.to(DEV)
+    gd = None if gain is None else gain.to(DEV)
+    codes, scale = tb.bitnet_act_quant(Xd, gain=gd, eps=1e-5, fwht=fwht, mode=mode)
+    X32 = X.float().numpy()
+    g32 = None if gain is None else gain.numpy()
+    q_ref, s_ref = ref.act_quant(X32, g32, 1e-5, fwht, MODES[mode])
+    sh = ref.shadow(X32, g32, 1e-5, fwht, MODES[mode])
+    label = f"M={M} K={K} fwht={fwht} {mode} {xdtype} gain={use_gain}"
+    parity.check_codes(host(codes), q_ref, sh, label)
+    parity.check_scale(host(scale), s_ref, label)
+
+
+@pytest.mark.parametrize("K", FWHT_K)
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_act_quant_fwht(K, mode):
+    _act_case(7, K, True, mode, "f32", False)
+
+
+@pytest.mark.parametrize("K", PLAIN_K)
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_act_quant_plain(K, mode):
+    _act_case(5, K, False, mode, "f32", False)
+
+
+@pytest.mark.parametrize("fwht", [True, False])
+def test_act_quant_bf16_and_gain(fwht):
+    _act_case(9, 4096, fwht, "int8", "bf16", True)
+    _act_case(3, 1024, fwht, "int4", "f32", True)
+
+
+def test_act_quant_many_tokens_flip_rate():
+    # 512 tokens x 8192: the flip-rate bound is statistical, so test it on a large sample
+    _act_case(512, 8192, True, "int4", "f32", False, seed=11)
+    _act_case(512, 8192, True, "int8", "f32", False, seed=12)
+
+
+def test_act_quant_zero_and_constant_tokens():
+    X = torch.zeros((4, 1024))
+    X[1] = 3.0
+    X[2, 5] = -7.0
+    for fwht in (True, False):
+        for mode in ("int8", "int4"):
+            codes, scale = tb.bitnet_act_quant(X.to(DEV), fwht=fwht, mode=mode)
+            q_ref, s_ref = ref.act_quant(X.numpy(), None, 1e-5, fwht, MODES[mode])
+            sh = ref.shadow(X.numpy(), None, 1e-5, fwht, MODES[mode])
+            parity.check_codes(host(codes), q_ref, sh, f"special rows fwht={fwht} {mode}")
+            assert np.all(host(codes)[0] == 0) and host(scale)[0] == 0
+
+
+# ----------------------------------------------------------------------------- GEMM on given codes
+GEMM_SHAPES = [
+    # decode kernel (M <= 16)
+    (1, 64, 128), (2, 100, 384), (5, 700, 2560), (8, 6912, 2560), (8, 2560, 6912), (9, 130, 640),
+    (16, 512, 1024),
+    # tcgen05 kernel
+    (17, 256, 128), (128, 256, 256), (130, 300, 384), (256, 520, 1024), (300, 1000, 2048),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_gemm_exact_accumulators(M, N, K, mode):
+    rng = np.random.default_rng(M * 1000003 + N * 7 + K)
+    lo, hi = (-128, 128) if mode == "int8" else (-8, 8)
+    q = rng.integers(lo, hi, size=(M, K)).astype(np.int8)
+    t = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = ref.pack(t)
+    scale = rng.uniform(0.1, 10.0, size=M).astype(np.float32)
+    alpha = np.array([0.0173], dtype=np.float32)
+    acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    out = tb.bitnet_ternary_gemm(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, acc_out=acc)
+    acc_ref = ref.gemm_packed(q, packed, N)
+    np.testing.assert_array_equal(host(acc), acc_ref)
+    out_ref = ref.dequant(acc_ref, scale, alpha[0], MODES[mode])
+    np.testing.assert_array_equal(host(out), out_ref)
+
+
+def test_gemm_extreme_codes():
+    # every code at the int8 extremes, every weight +1/-1: |acc| = 128 K is the largest possible
+    for M, N, K in [(4, 64, 16384), (32, 256, 16384)]:
+        q = np.full((M, K), -128, np.int8)
+        q[::2] = 127
+        t = np.ones((N, K), np.int8)
+        t[1::3] = -1
+        packed = ref.pack(t)
+        scale = np.ones(M, np.float32)
+        alpha = np.ones(1, np.float32)
+        acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+        tb.bitnet_ternary_gemm(dev(q), dev(scale), "int8", dev(packed), dev(alpha), N, acc_out=acc)
+        np.testing.assert_array_equal(host(acc), ref.gemm_packed(q, packed, N))
+
+
+# ----------------------------------------------------------------------------- whole forward
+def _forward_case(case, sample_rows=None):
+    Xd = case.X.to(DEV)
+    W = case.W.to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(W, eps=case.eps)
+    out = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, case.N, eps=case.eps, fwht=case.fwht, mode=case.mode)
+    codes, _ = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=case.fwht, mode=case.mode)
+    torch.cuda.synchronize()
+    rows = np.arange(case.M) if sample_rows is None else sample_rows
+    X32 = case.X.float().numpy()[rows]
+    p_ref, a_ref, _ = ref.pack_weights(case.W.numpy(), eps=case.eps)
+    assert host(alpha)[0] == a_ref
+    np.testing.assert_array_equal(host(packed), p_ref)
+    mode = MODES[case.mode]
+    r = ref.hbitlinear_forward(X32, p_ref, a_ref, case.N, eps=case.eps, fwht_on=case.fwht, mode=mode)
+    sh = ref.shadow(X32, None, case.eps, case.fwht, mode)
+    gcodes = host(codes)[rows]
+    parity.check_codes(gcodes, r.codes, sh, case.name)
+    gout = host(out)[rows]
+    # same codes -> same output (up to the per-token scale's last bits)
+    out_same = ref.dequant(ref.gemm_packed(gcodes, p_ref, case.N), r.scale_x, a_ref, mode)
+    parity.check_out_same_codes(gout, out_same, case.name)
+    parity.check_out_end_to_end(gout, r.out, gcodes, r.codes, r.scale_x, a_ref, mode, case.name)
+
+
+def test_forward_tiny_int8_fwht():
+    _forward_case(synthetic.tiny_hbitlinear())
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+@pytest.mark.parametrize("NK", [(6912, 2560), (2560, 6912)])
+def test_forward_decode_full_size(M, NK):
+    _forward_case(synthetic.decode(M, N=NK[0], K=NK[1]))
+
+
+@pytest.mark.parametrize("M,K,N,mode,fwht,xdt", [
+    (3, 1024, 200, "int4", True, "f32"),
+    (13, 512, 520, "int8", True, "bf16"),
+    (100, 1024, 300, "int4", True, "f32"),
+    (257, 2048, 520, "int8", False, "bf16"),
+    (384, 4096, 768, "int4", True, "f32"),
+])
+def test_forward_ragged(M, K, N, mode, fwht, xdt):
+    case = synthetic.make_case("ragged", M, K, N, x_kind="student_t3", outliers=max(1, K // 100),
+                               outlier_gain=50.0, x_dtype=xdt, fwht=fwht, mode=mode, seed=M + K)
+    _forward_case(case)
+
+
+def _sample(M, n=32, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, n - 2, replace=False)]))
+    return rows
+
+
+def test_forward_wdown_int4_full_size_sampled():
+    case = synthetic.wdown_int4()  # M=2048, K=8192, N=2048, Student-t + 1% outliers x50
+    _forward_case(case, _sample(case.M))
+
+
+@pytest.mark.parametrize("N,fwht", [(4096, True), (11008, False)])
+def test_forward_prefill_bf16_full_size_sampled(N, fwht):
+    case = synthetic.prefill_int8(M=4096, K=4096, N=N, fwht=fwht)
+    _forward_case(case, _sample(case.M, 24))
+
+
+@pytest.mark.parametrize("M,K", [(1, 16384), (8, 4096), (64, 16384), (512, 4096), (8192, 16384)])
+def test_forward_msweep_int4_sampled(M, K):
+    case = synthetic.msweep_int4(M, K)
+    _forward_case(case, None if M <= 64 else _sample(M, 16))
+
+
+# ----------------------------------------------------------------------------- properties
+def test_forward_deterministic_and_graph_capturable():
+    case = synthetic.msweep_int4(64, 4096, N=1024, seed=3)
+    Xd = case.X.to(DEV)
+    layer = tb.HBitLinear(case.W.to(DEV), mode="int4", fwht=True)
+    o1 = layer(Xd).clone()
+    o2 = layer(Xd).clone()
+    assert torch.equal(o1, o2)
+    out = torch.empty_like(o1)
+    layer.workspace(Xd.shape[0], Xd.device)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer(Xd, out=out)  # warm (attribute caches) outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer(Xd, out=out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, o1)
+
+
+def test_empty_batch_and_errors():
+    W = synthetic.gaussian((64, 256), 0.02, synthetic.generator(1)).to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(W)
+    X = torch.empty((0, 256), device=DEV)
+    out = tb.bitnet_hbitlinear_forward(X, packed, alpha, 64)
+    assert out.shape == (0, 64)
+    with pytest.raises(tb.BitnetError) as e:
+        tb.bitnet_act_quant(torch.ones((2, 2560), device=DEV), fwht=True)
+    assert e.value.status == 3
+    with pytest.raises(tb.BitnetError):
+        tb.bitnet_act_quant(torch.ones((2, 200), device=DEV), fwht=False)
+
+
+def test_timeout_path_reports_and_recovers():
+    tb.bitnet_selftest_wait_timeout(2000)
+    assert tb.bitnet_get_last_device_status() == 5
+    assert tb.bitnet_get_last_device_status() == 0
+    # the context is still usable afterwards
+    x = torch.ones((2, 256), device=DEV)
+    codes, scale = tb.bitnet_act_quant(x, fwht=True)
+    torch.cuda.synchronize()
+    assert host(codes)[0, 0] == 127
