@@ -155,6 +155,36 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype
                                           void *ws, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
+ * bitnet_hbitlinear_forward_noalloc -- the same forward as bitnet_hbitlinear_forward,
+ * for callers that cannot allocate device memory: a plugin or extension interface
+ * that hands a kernel only its input and output buffers, a runtime that owns all
+ * device memory in a preplanned arena, or a latency-critical path that must never
+ * reach cudaMalloc (which can synchronise the device).  The paper has no
+ * counterpart; this is a deployment variant of the entry point above.
+ *   Arguments and results are those of bitnet_hbitlinear_forward without ws/ws_bytes.
+ *   The codes and scales between the two kernels live in a fixed array of
+ *   BITNET_NOALLOC_SCRATCH_BYTES in the library's own device memory; every GPU that
+ *   loads the library holds that array until the process exits.  A call needs
+ *   bitnet_forward_workspace_bytes(M, K) <= BITNET_NOALLOC_SCRATCH_BYTES (4 MiB:
+ *   for example M*K up to about 4.19 million); larger calls return
+ *   BITNET_ERR_WORKSPACE without launching anything.
+ *   The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *   routine).  Its first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.
+ *   All calls on a device share the one array, which keeps the last call's
+ *   contents (nothing in it needs clearing: every code and scale read is first
+ *   written by the same call).  Calls that overlap on the GPU -- on different
+ *   streams without ordering between them -- race on the array; order them.
+ * ------------------------------------------------------------------------ */
+#define BITNET_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitnet_dtype_t xdt, int64_t M,
+                                                              int64_t K, const float *gain, float eps, int fwht,
+                                                              bitnet_act_mode_t mode, const uint8_t *packed,
+                                                              const float *alpha, int64_t N, float *out,
+                                                              void *stream);
+
+/* --------------------------------------------------------------------------
  * Status and diagnostics (no counterpart on the pages).
  * bitnet_status_string: static English text for a status code.
  * bitnet_get_last_device_status: synchronises `stream`, returns the status word

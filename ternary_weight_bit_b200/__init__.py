@@ -23,7 +23,7 @@ from ._native import BitnetError
 
 __all__ = [
     "BitnetError", "HBitLinear", "bitnet_pack_ternary", "bitnet_act_quant", "bitnet_ternary_gemm",
-    "bitnet_hbitlinear_forward", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
+    "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
 ]
 
@@ -157,6 +157,28 @@ def bitnet_hbitlinear_forward(X: torch.Tensor, packed: torch.Tensor, alpha: torc
                   L.bitnet_hbitlinear_forward(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)),
                                               mode_id(mode), _ptr(packed), _ptr(alpha), N, _ptr(out), _ptr(ws),
                                               ws.numel(), _stream(stream)))
+    return out
+
+
+def bitnet_hbitlinear_forward_noalloc(X: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, N: int,
+                                      gain=None, eps: float = 1e-5, fwht: bool = True, mode="int8", out=None,
+                                      stream=None):
+    """The forward without a caller workspace, for callers that cannot allocate device memory
+    (the scratch is a fixed 4 MiB array inside the library; see include/bitnet.h)."""
+    L = _native.load()
+    _need(X, "X")
+    M, K = X.shape
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(alpha, "alpha", torch.float32)
+    if gain is not None:
+        _need(gain, "gain", torch.float32, (K,))
+    if out is None:
+        raise ValueError("out must be given: this entry point is for callers that cannot allocate")
+    _need(out, "out", torch.float32, (M, N))
+    _native.check("bitnet_hbitlinear_forward_noalloc",
+                  L.bitnet_hbitlinear_forward_noalloc(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)),
+                                                      mode_id(mode), _ptr(packed), _ptr(alpha), N, _ptr(out),
+                                                      _stream(stream)))
     return out
 
 

@@ -39,7 +39,6 @@ bitnet_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK :
 
 constexpr int64_t kMaxK = 32768;
 constexpr int64_t kMaxRows = (int64_t)1 << 30;  // M and N bounds (TMA coordinates are int32)
-constexpr int kGemvMaxM = 16;
 
 bitnet_status_t check_k(int64_t K, int fwht) {
     if (K <= 0 || K % 128 != 0 || K > kMaxK) return BITNET_ERR_UNSUPPORTED_SHAPE;

@@ -7,6 +7,10 @@
 
 namespace bitnet {
 
+// Forwards and GEMMs with at most this many tokens run the decode kernel (gemv.cu);
+// larger ones the tcgen05 GEMM (gemm_sm100.cu).
+constexpr int kGemvMaxM = 16;
+
 // Encode a 2-D tiled TMA descriptor over a row-major byte matrix [rows][row_bytes]
 // (element type uint8).  box = {box_x bytes, box_y rows}; swizzle is one of
 // CU_TENSOR_MAP_SWIZZLE_{NONE,32B,64B,128B}.  Out-of-bounds boxes read as zero.
