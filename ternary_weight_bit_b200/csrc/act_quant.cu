@@ -164,7 +164,9 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
     extern __shared__ __align__(16) float sm[];  // K floats
     __shared__ float red[32];
 
-    pdl_launch_dependents();  // the GEMM may start streaming weights now
+    // X may come from the previous kernel: wait for it, then let the GEMM start streaming weights.
+    pdl_wait_prerequisites();
+    pdl_launch_dependents();
 
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(T)
 act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gain, int K, float eps,
                        int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x) {
     __shared__ float red[32];
+    pdl_wait_prerequisites();
     pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
@@ -329,6 +332,24 @@ act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gai
     if (tid == 0) scale_x[blockIdx.x] = stat;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel of the stream finishes; it waits (griddepcontrol.wait) before
+// reading anything, and only then lets its own dependents start.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int LOGK, bool BF16>
 cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
                         float *scale_x, cudaStream_t s) {
@@ -346,16 +367,15 @@ cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, 
             if (dev < kMaxDevices) done[dev] = true;
         }
     }
-    kern<<<(unsigned)M, S::T, smem, s>>>(X, gain, eps, mode, codes, scale_x);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, X, gain, eps, mode, codes, scale_x);
 }
 
 template <int NV, bool BF16>
 cudaError_t launch_plain(const void *X, int64_t M, int K, const float *gain, float eps, int mode,
                          int8_t *codes, float *scale_x, cudaStream_t s) {
     constexpr int T = 256;
-    act_quant_plain_kernel<T, NV, BF16><<<(unsigned)M, T, 0, s>>>(X, gain, K, eps, mode, codes, scale_x);
-    return cudaGetLastError();
+    return launch_pdl(act_quant_plain_kernel<T, NV, BF16>, dim3((unsigned)M), dim3(T), 0, s, X, gain, K, eps, mode,
+                      codes, scale_x);
 }
 
 template <bool BF16>

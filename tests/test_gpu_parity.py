@@ -130,7 +130,8 @@ GEMM_SHAPES = [
     (1, 64, 128), (2, 100, 384), (5, 700, 2560), (8, 6912, 2560), (8, 2560, 6912), (9, 130, 640),
     (16, 512, 1024),
     # tcgen05 kernel
-    (17, 256, 128), (128, 256, 256), (130, 300, 384), (256, 520, 1024), (300, 1000, 2048),
+    (17, 256, 128), (64, 200, 640), (128, 256, 256), (130, 300, 384), (256, 520, 1024), (300, 1000, 2048),
+    (1200, 2560, 128),  # large enough for the 256-token tile
 ]
 
 
