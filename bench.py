@@ -110,7 +110,8 @@ def load_peaks():
 
 
 def profile_traffic(kernel_key: str, source_file: str):
-    """Per-launch DRAM bytes from the committed ncu summary, if the kernel is unchanged since."""
+    """Per-launch DRAM bytes of the dominant kernel on this workload, from the committed ncu
+    summary profiles/<kernel_key>.md, if the kernel source is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", f"{kernel_key}.md")
     try:
         text = open(path).read()
@@ -394,7 +395,7 @@ def run_ours(args):
         peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic("gemv_decode_traffic", "gemv.cu"),
+                "traffic": profile_traffic(f"gemv_traffic_{args.workload}", "gemv.cu"),
                 "kernel": "gemv_kernel (register-streamed packed weights, mma.sync s8, in-CTA split-K)",
                 "peak_source": f"hbm_gbs of {peak_src} MEASURED_PEAKS.json (copy, burst)",
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
@@ -405,7 +406,7 @@ def run_ours(args):
         peak = 2.0 * bf16
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic("gemm_tc_traffic", "gemm_sm100.cu"),
+                "traffic": profile_traffic(f"gemm_tc_traffic_{args.workload}", "gemm_sm100.cu"),
                 "kernel": "gemm_tc_kernel (tcgen05 kind::i8, weights as TMEM A operand, TMEM accumulator)",
                 "peak_source": f"int8 dense = 2 x bf16_tflops of {peak_src} MEASURED_PEAKS.json (nominal ratio)",
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
