@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 1
+#define BITNET_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -130,8 +130,10 @@ BITNET_API bitnet_status_t bitnet_act_quant(const void *X, bitnet_dtype_t xdt, i
  *   alpha    one fp32, device, read only.
  *   out      [M][N] fp32, device, written.
  *   acc_out  [M][N] int32, device, written when not NULL (for exactness checks).
- * M <= 16 runs the weight-streaming decode kernel (tensor-core mma.sync, cluster
- * split-K); larger M runs the tcgen05 int8 tensor-core GEMM with TMEM accumulators.
+ * M <= 16 runs the weight-streaming decode kernel (tensor-core mma.sync, split-K
+ * over the warps of a CTA); larger M runs the persistent tcgen05 int8 tensor-core
+ * GEMM with TMEM accumulators, whose token-tile size is chosen per shape (see
+ * bitnet_gemm_token_tile below).
  * ------------------------------------------------------------------------ */
 BITNET_API bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x,
                                     bitnet_act_mode_t mode, const uint8_t *packed,
@@ -183,6 +185,22 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
                                                               bitnet_act_mode_t mode, const uint8_t *packed,
                                                               const float *alpha, int64_t N, float *out,
                                                               void *stream);
+
+/* --------------------------------------------------------------------------
+ * Prefill GEMM tile control (no counterpart on the pages).
+ * bitnet_gemm_token_tile: the token-tile size (256, 224, 192, 128 or 64 tokens
+ *   per tensor-core tile) that bitnet_ternary_gemm and the forwards use for an
+ *   M x N x K problem on the current device; 0 when M <= 16 (the decode kernel
+ *   runs instead); -1 for sizes the GEMM rejects.  Includes any forced value.
+ * bitnet_gemm_force_token_tile: process-wide override of that choice, for every
+ *   device and thread: 0 restores the automatic choice; 256, 224, 192, 128 or 64
+ *   forces it; any other value returns BITNET_ERR_INVALID_ARG and changes nothing.
+ *   Results do not depend on the tile (the int32 accumulators are exact and the
+ *   epilogue is elementwise), only the speed does.  For tests and tuning; set it
+ *   while no other thread is launching GEMMs.
+ * ------------------------------------------------------------------------ */
+BITNET_API int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K);
+BITNET_API bitnet_status_t bitnet_gemm_force_token_tile(int token_tile);
 
 /* --------------------------------------------------------------------------
  * Status and diagnostics (no counterpart on the pages).

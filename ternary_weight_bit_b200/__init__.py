@@ -25,6 +25,7 @@ __all__ = [
     "BitnetError", "HBitLinear", "bitnet_pack_ternary", "bitnet_act_quant", "bitnet_ternary_gemm",
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
+    "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile",
 ]
 
 _MODES = {"int8": _native.ACT_INT8_ABSMAX, "int4": _native.ACT_INT4_ABSMEAN}
@@ -63,6 +64,16 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None) -> None:
 
 def bitnet_abi_version() -> int:
     return _native.load().bitnet_abi_version()
+
+
+def bitnet_gemm_token_tile(M: int, N: int, K: int) -> int:
+    """Token-tile size of the tcgen05 GEMM for this shape (0: decode kernel, -1: rejected)."""
+    return _native.load().bitnet_gemm_token_tile(M, N, K)
+
+
+def bitnet_gemm_force_token_tile(token_tile: int) -> None:
+    """Force the GEMM token tile (256/224/192/128/64) process-wide; 0 restores the automatic choice."""
+    _native.check("bitnet_gemm_force_token_tile", _native.load().bitnet_gemm_force_token_tile(token_tile))
 
 
 def bitnet_pack_workspace_bytes(N: int, K: int) -> int:

@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_get_last_device_status": (I, [P]),
         "bitnet_selftest_wait_timeout": (I, [U32, P]),
         "bitnet_abi_version": (I, []),
+        "bitnet_gemm_token_tile": (I, [I64, I64, I64]),
+        "bitnet_gemm_force_token_tile": (I, [I]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)

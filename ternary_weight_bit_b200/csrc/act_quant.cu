@@ -74,6 +74,19 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
     return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
+// As quant_byte, but returns the whole rounded word (code in the low byte) and
+// clips only when asked.
+__device__ __forceinline__ uint32_t quant_bits(float y, float s, float lo, float hi, bool clip) {
+    float v = __fmul_rn(y, s);
+    if (clip) v = fminf(fmaxf(v, lo), hi);
+    return __float_as_uint(__fadd_rn(v, 12582912.0f));
+}
+
+// Low bytes of four words -> one word (byte permutes).
+__device__ __forceinline__ uint32_t pack4_perm(uint32_t f0, uint32_t f1, uint32_t f2, uint32_t f3) {
+    return __byte_perm(__byte_perm(f0, f1, 0x0040), __byte_perm(f2, f3, 0x0040), 0x5410);
+}
+
 struct QuantParams {
     float s, lo, hi;
 };
@@ -139,21 +152,31 @@ struct FwhtShape {
     static constexpr int PHASES = (LOGK + ELOG - 1) / ELOG;
 };
 
-// Index of register r of thread tid in phase p: the register bits are
-// [lo, lo+nb) plus, in a short last phase, the low `pass` bits as passengers.
+// Index of register r of thread tid in phase p is tid_part(p, tid) | reg_part(p, r):
+// the register bits are [lo, lo+nb) plus, in a short last phase, the low `pass`
+// bits as passengers; the thread bits fill the rest.  The two parts occupy
+// disjoint bits, so their padded addresses add up (see pad()).
 template <int LOGK, int ELOG>
-__device__ __forceinline__ int phase_index(int p, int tid, int r) {
+__device__ __forceinline__ int tid_part(int p, int tid) {
     const int lo = p * ELOG;
     const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
     const int pass = ELOG - nb;
     const int tl = lo - pass;
-    const int r_pass = r & ((1 << pass) - 1);
-    const int r_hi = r >> pass;
-    return r_pass | ((tid & ((1 << tl) - 1)) << pass) | (r_hi << lo) | ((tid >> tl) << (lo + nb));
+    return ((tid & ((1 << tl) - 1)) << pass) | ((tid >> tl) << (lo + nb));
+}
+template <int LOGK, int ELOG>
+__device__ __forceinline__ int reg_part(int p, int r) {
+    const int lo = p * ELOG;
+    const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
+    const int pass = ELOG - nb;
+    return (r & ((1 << pass) - 1)) | ((r >> pass) << lo);
 }
 
-// Bank-spreading permutation of the shared-memory copy of a token.
-__device__ __forceinline__ int swz(int i) { return i ^ ((i >> 5) & 31); }
+// Shared-memory position of element i: one pad word after every 32 elements
+// spreads the strided phase accesses over the banks.  For disjoint bit fields
+// a, b: pad(a | b) = pad(a) + pad(b), so every register's address is a
+// compile-time offset from one per-thread base.
+__device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
 
 template <int LOGK, bool BF16>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::T)
@@ -161,7 +184,7 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
                       int8_t *__restrict__ codes, float *__restrict__ scale_x) {
     using S = FwhtShape<LOGK>;
     constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
-    extern __shared__ __align__(16) float sm[];  // K floats
+    extern __shared__ __align__(16) float sm[];  // K + K/32 floats (padded)
     __shared__ float red[32];
 
     // X may come from the previous kernel: wait for it, then let the GEMM start streaming weights.
@@ -196,11 +219,13 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
     for (int p = 0; p < P; ++p) {
         if (p > 0) {
             __syncthreads();
+            float *wb = sm + pad(tid_part<LOGK, ELOG>(p - 1, tid));
 #pragma unroll
-            for (int r = 0; r < E; ++r) sm[swz(phase_index<LOGK, ELOG>(p - 1, tid, r))] = v[r];
+            for (int r = 0; r < E; ++r) wb[pad(reg_part<LOGK, ELOG>(p - 1, r))] = v[r];
             __syncthreads();
+            const float *rb = sm + pad(tid_part<LOGK, ELOG>(p, tid));
 #pragma unroll
-            for (int r = 0; r < E; ++r) v[r] = sm[swz(phase_index<LOGK, ELOG>(p, tid, r))];
+            for (int r = 0; r < E; ++r) v[r] = rb[pad(reg_part<LOGK, ELOG>(p, r))];
         }
         const int lo = p * ELOG;
         const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
@@ -244,26 +269,26 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
         stat = __fdiv_rn(block_sum<T>(sa, red), (float)K);
     }
     const QuantParams q = quant_params(stat, eps, mode);
+    // int8: |y| <= gamma makes |y*s| < 127.5, so the clip can never act.
+    const bool clip = mode != BITNET_ACT_INT8_ABSMAX;
 
     // Store the codes in the last phase's layout.
     constexpr int LASTLO = (P - 1) * ELOG;
     constexpr int LASTNB = (LOGK - LASTLO) < ELOG ? (LOGK - LASTLO) : ELOG;
     constexpr int LASTPASS = ELOG - LASTNB;
-    int8_t *out = codes + row;
+    int8_t *out = codes + row + tid_part<LOGK, ELOG>(P - 1, tid);
     if constexpr (LASTPASS >= 2) {
 #pragma unroll
         for (int r = 0; r < E; r += 4) {
-            const int i = phase_index<LOGK, ELOG>(P - 1, tid, r);
-            const uint32_t w = pack4(quant_byte(v[r], q.s, q.lo, q.hi), quant_byte(v[r + 1], q.s, q.lo, q.hi),
-                                     quant_byte(v[r + 2], q.s, q.lo, q.hi), quant_byte(v[r + 3], q.s, q.lo, q.hi));
-            *reinterpret_cast<uint32_t *>(out + i) = w;
+            uint32_t f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = quant_bits(v[r + e], q.s, q.lo, q.hi, clip);
+            *reinterpret_cast<uint32_t *>(out + reg_part<LOGK, ELOG>(P - 1, r)) = pack4_perm(f[0], f[1], f[2], f[3]);
         }
     } else {
 #pragma unroll
-        for (int r = 0; r < E; ++r) {
-            const int i = phase_index<LOGK, ELOG>(P - 1, tid, r);
-            out[i] = (int8_t)quant_byte(v[r], q.s, q.lo, q.hi);
-        }
+        for (int r = 0; r < E; ++r)
+            out[reg_part<LOGK, ELOG>(P - 1, r)] = (int8_t)(quant_bits(v[r], q.s, q.lo, q.hi, clip) & 0xFFu);
     }
     if (tid == 0) scale_x[blockIdx.x] = stat;
 }
@@ -354,7 +379,7 @@ template <int LOGK, bool BF16>
 cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
                         float *scale_x, cudaStream_t s) {
     using S = FwhtShape<LOGK>;
-    const size_t smem = (size_t)S::K * sizeof(float);
+    const size_t smem = (size_t)(S::K + S::K / 32) * sizeof(float);
     auto kern = act_quant_fwht_kernel<LOGK, BF16>;
     if (smem > 48 * 1024) {
         static bool done[kMaxDevices] = {};

@@ -63,6 +63,19 @@ bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_x,
+                      uint32_t box_y) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {box_x, box_y};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int *device_status_ptr() {
     static int *ptrs[kMaxDevices] = {};
     int dev = 0;
@@ -224,6 +237,16 @@ bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int
     cudaError_t e = launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, nullptr, true, s));
+}
+
+int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 1 || N > kMaxRows || check_k(K, 0) != BITNET_OK) return -1;
+    if (M <= kGemvMaxM) return 0;
+    return gemm_pick_tile((int)M, (int)N, (int)K, sm_count());
+}
+
+bitnet_status_t bitnet_gemm_force_token_tile(int token_tile) {
+    return gemm_force_tile(token_tile) ? BITNET_OK : BITNET_ERR_INVALID_ARG;
 }
 
 bitnet_status_t bitnet_get_last_device_status(void *stream) {

@@ -1,5 +1,5 @@
 // gemm_sm100.cu -- prefill path of steps 4b-5 on the 5th-generation tensor cores:
-// tcgen05.mma kind::i8 (int8 x int8 -> int32) with the accumulator in TMEM.
+// tcgen05.mma kind::i8 (int8 x int8 -> int32) with the accumulators in TMEM.
 //
 // Method: bitnet_v2_engine.py page, HBitLinear.forward (F.linear of the quantised
 // activations and ternary weights); BitLinear_b158.forward in the youngju.dev BitNet
@@ -11,16 +11,30 @@
 //   B = BT activation-code rows (tokens), TMA-loaded into shared memory in the
 //       K-major 128-byte-swizzled layout;
 //   D = 128 lanes (weight rows) x BT int32 columns (tokens) in TMEM.
-// Per 128-k stage the shared memory only carries the activation tile (BT x 128 B)
+// Per 128-k stage the shared memory carries only the activation tile (BT x 128 B)
 // and the packed weights (128 x 32 B).
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer (activation tile, 128B swizzle; packed weights, 32B swizzle)
-//   warp 1     TMEM allocator; lane 0 issues 4 x tcgen05.mma per stage and the commits
-//   warps 2-5  each owns the 32 TMEM lanes (weight rows) of its lane quarter: unpack
-//              its rows into the stage's A columns, then run the epilogue
-//              (tcgen05.ld, out[m][n] = acc * f[m], stores coalesced along n).
+// Persistent: one CTA per SM walks the output tiles (weight-row block fastest, so
+// an activation tile is reused from L2 by consecutive tiles).  Three rings keep the
+// roles decoupled:
+//   ST shared-memory stages  TMA -> unpack + MMA; freed by the MMA commit
+//   AS TMEM weight slots     unpack -> MMA (32 columns = 128 k each); freed by the MMA commit
+//   DB accumulator buffers   MMA -> epilogue; freed by the epilogue after tcgen05.ld
+// With DB = 2 the epilogue of one tile overlaps the MMAs of the next; with DB = 1
+// (BT = 256 fills TMEM) the MMAs of the next tile wait for the drain, while the
+// TMA and unpack rings run on.
+//
+// Warp roles (64 + 128 UW + 128 threads):
+//   warp 0       TMA producer; the whole warp runs the loop, an elected lane issues
+//   warp 1       TMEM allocator and MMA issuer (4 x tcgen05.mma per stage, commits),
+//                likewise warp-uniform with elected issue
+//   UW sets of 4 unpack warps; set u takes the stages it with it % UW == u.  Warp w
+//                owns TMEM lanes 32 (w % 4) .. +31 (= weight rows) of its slot.
+//   4 epilogue warps: tcgen05.ld, out[m][n] = acc * f[m]; the fp32 tile goes out
+//                through shared memory with one TMA bulk tensor store per 32 tokens.
 // All waits are bounded; a timeout is recorded in the device status word.
+#include <string.h>
+
 #include "common.cuh"
 #include "host.h"
 
@@ -28,32 +42,44 @@ namespace bitnet {
 
 namespace {
 
-constexpr int BW = 128;  // weight rows per tile (MMA M)
-constexpr int BK = 128;  // k per stage
-constexpr int THREADS = 192;
+constexpr int BW = 128;         // weight rows per tile (MMA M)
+constexpr int BK = 128;         // k per stage
+constexpr int OUT_TOKENS = 32;  // tokens per output store box
 
-template <int BT>
+template <int BT_, int ST_, int AS_, int DB_, int UW_>
 struct TcCfg {
-    static constexpr int STAGES = BT >= 256 ? 4 : 6;
-    static constexpr int CTAS_PER_SM = BT <= 64 ? 2 : 1;
-    static constexpr int B_BYTES = BT * BK;        // activation tile
-    static constexpr int P_BYTES = BW * BK / 4;    // packed weight tile (4 KB)
+    static constexpr int BT = BT_, ST = ST_, AS = AS_, DB = DB_, UW = UW_;
+    static constexpr int THREADS = 64 + 128 * UW + 128;
+    static constexpr int B_BYTES = BT * BK;      // activation tile
+    static constexpr int P_BYTES = BW * BK / 4;  // packed weight tile (4 KB)
     static constexpr int B_OFF = 0;
-    static constexpr int P_OFF = STAGES * B_BYTES;
-    static constexpr int F_OFF = P_OFF + STAGES * P_BYTES;  // per-token dequant factors
-    static constexpr int BAR_OFF = F_OFF + BT * 4;
-    static constexpr int NUM_BARS = 3 * STAGES + 1;
+    static constexpr int P_OFF = ST * B_BYTES;
+    static constexpr int O_OFF = P_OFF + ST * P_BYTES;             // 2 x [32 tokens][128 rows] fp32
+    static constexpr int F_OFF = O_OFF + 2 * OUT_TOKENS * BW * 4;  // per-token dequant factors, DB rows
+    static constexpr int BAR_OFF = F_OFF + DB * BT * 4;
+    static constexpr int NUM_BARS = 2 * ST + 2 * AS + 2 * DB;
     static constexpr int TMEM_SLOT_OFF = BAR_OFF + NUM_BARS * 8;
-    static constexpr int SMEM = TMEM_SLOT_OFF + 16 + 1024;
-    // D: BT columns, A stages: 32 columns each; allocations are powers of two.
-    static constexpr uint32_t TMEM_COLS = (BT + 32 * STAGES) <= 256 ? 256 : 512;
-    static constexpr uint32_t A_COL0 = BT;
-    static_assert(BT + 32 * STAGES <= (int)TMEM_COLS, "TMEM budget");
-    static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "co-resident CTAs must fit in TMEM together");
+    static constexpr int SMEM_USED = TMEM_SLOT_OFF + 16 + 1024;  // + alignment slack
+    // At least 120 KB so that two CTAs never share an SM (each allocates all of TMEM).
+    static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t A_COL0 = DB * BT;  // D buffers first, then the weight slots
+    static_assert(BT % 32 == 0 && BT >= 64 && BT <= 256, "MMA N");
+    static_assert(DB * BT + 32 * AS <= 512, "TMEM budget");
+    static_assert(SMEM_USED <= 232448, "shared memory budget");
+    static_assert(UW <= ST && UW <= AS, "each unpack set advances by UW stages");
+    static_assert(B_BYTES % 1024 == 0, "128B-swizzled tiles stay 1024-byte aligned");
     // D = s32, A = s8, B = s8, K-major both, N = BT, M = 128.
     static constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) |
                                       ((uint32_t)(BW >> 4) << 24);
 };
+
+// The configurations the dispatcher chooses from.
+using Cfg256 = TcCfg<256, 5, 4, 1, 2>;
+using Cfg224 = TcCfg<224, 5, 2, 2, 2>;
+using Cfg192 = TcCfg<192, 6, 4, 2, 2>;
+using Cfg128 = TcCfg<128, 8, 8, 2, 2>;
+using Cfg64 = TcCfg<64, 12, 8, 2, 2>;
 
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     uint64_t d = 0;
@@ -71,17 +97,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     return v;
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, int8 x int8 -> int32.
-__device__ __forceinline__ void umma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -96,33 +111,51 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-template <int BT>
-__global__ void __launch_bounds__(THREADS, 1)
+// Tile t -> (weight-row block, token block); consecutive tiles walk the weight
+// blocks of one token block, so the activation tile stays hot in L2.
+struct TileMap {
+    int nb_blocks;
+    __device__ __forceinline__ void get(int t, int BT, int &n0, int &m0) const {
+        n0 = (t % nb_blocks) * BW;
+        m0 = (t / nb_blocks) * BT;
+    }
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w,
-               const float *__restrict__ scale_x, const float *__restrict__ alpha, int mode, int M, int N, int K,
-               float *__restrict__ out, int32_t *__restrict__ acc_out, int *status) {
-    using C = TcCfg<BT>;
+               const __grid_constant__ CUtensorMap tm_out, int tma_out, const float *__restrict__ scale_x,
+               const float *__restrict__ alpha, int mode, int M, int N, int K, float *__restrict__ out,
+               int32_t *__restrict__ acc_out, int *status) {
+    constexpr int BT = C::BT, ST = C::ST, AS = C::AS, DB = C::DB, UW = C::UW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-    uint64_t *unpacked = full + C::STAGES;
-    uint64_t *empty = unpacked + C::STAGES;
-    uint64_t *accfull = empty + C::STAGES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    // barrier i at bar_base + 8 i: full[ST], sfree[ST], unpacked[AS], afree[AS], accfull[DB], accempty[DB]
+    const uint32_t FULL = smem_u32(bars), SFREE = FULL + 8 * ST, UNPACKED = SFREE + 8 * ST,
+                   AFREE = UNPACKED + 8 * AS, ACCFULL = AFREE + 8 * AS, ACCEMPTY = ACCFULL + 8 * DB;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::TMEM_SLOT_OFF);
     float *fac = reinterpret_cast<float *>(smem + C::F_OFF);
+    const uint32_t sB0 = smem_u32(smem + C::B_OFF), sP0 = smem_u32(smem + C::P_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BW;  // weight rows
-    const int m0 = blockIdx.y * BT;  // tokens
     const int KB = K / BK;
+    const TileMap tmap{(N + BW - 1) / BW};
+    const int tiles = tmap.nb_blocks * ((M + BT - 1) / BT);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&unpacked[s], 4);
-            mbar_init(&empty[s], 1);
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(bars + i, 1);       // full: expect_tx arrival + TMA bytes
+            mbar_init(bars + ST + i, 1);  // sfree: MMA commit
         }
-        mbar_init(accfull, 1);
+        for (int i = 0; i < AS; ++i) {
+            mbar_init(bars + 2 * ST + i, 4);       // unpacked: the four warps of one set
+            mbar_init(bars + 2 * ST + AS + i, 1);  // afree: MMA commit
+        }
+        for (int i = 0; i < DB; ++i) {
+            mbar_init(bars + 2 * ST + 2 * AS + i, 1);       // accfull: MMA commit
+            mbar_init(bars + 2 * ST + 2 * AS + DB + i, 4);  // accempty: the four epilogue warps
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -139,106 +172,201 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         if (lane == 0) {
             tma_prefetch_desc(&tm_act);
             tma_prefetch_desc(&tm_w);
-            const int pre = KB < C::STAGES ? KB : C::STAGES;
-            for (int kb = 0; kb < pre; ++kb) {
-                mbar_arrive_expect_tx(&full[kb], C::B_BYTES + C::P_BYTES);
-                tma_load_2d(smem + C::P_OFF + kb * C::P_BYTES, &tm_w, &full[kb], kb * (BK / 4), n0);
-            }
-            pdl_wait_prerequisites();  // activation codes come from the previous kernel
-            for (int kb = 0; kb < pre; ++kb)
-                tma_load_2d(smem + C::B_OFF + kb * C::B_BYTES, &tm_act, &full[kb], kb * BK, m0);
-            int issued = pre;
-            for (int kb = C::STAGES; kb < KB; ++kb) {
-                const int s = kb % C::STAGES;
-                if (!mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1, status)) break;
-                mbar_arrive_expect_tx(&full[s], C::B_BYTES + C::P_BYTES);
-                tma_load_2d(smem + C::P_OFF + s * C::P_BYTES, &tm_w, &full[s], kb * (BK / 4), n0);
-                tma_load_2d(smem + C::B_OFF + s * C::B_BYTES, &tm_act, &full[s], kb * BK, m0);
-                issued = kb + 1;
-            }
-            const int last = issued - 1;  // every issued load must land before exit
-            for (int s = 0; s < C::STAGES && s <= last; ++s) {
-                const int li = last - ((last - s) % C::STAGES);
-                mbar_wait(&full[s], (li / C::STAGES) & 1, status);
-            }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        __syncwarp();
+        bool waited = false, ok = true, wrapped = false;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            int n0, m0;
+            tmap.get(t, BT, n0, m0);
             for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % C::STAGES;
-                const uint32_t par = (kb / C::STAGES) & 1;
-                if (!mbar_wait(&full[s], par, status)) break;
-                if (!mbar_wait(&unpacked[s], par, status)) break;
-                tc_fence_after();
-                const uint64_t bdesc = smem_desc_sw128(smem_u32(smem + C::B_OFF + s * C::B_BYTES));
-                const uint32_t a_tmem = tmem_base + C::A_COL0 + 32 * s;
-#pragma unroll
-                for (int j = 0; j < BK / 32; ++j)  // K = 32 per MMA: 8 TMEM columns of A, 32 bytes of B rows
-                    umma_i8_ts(tmem_base, a_tmem + 8 * j, bdesc + (uint64_t)(2 * j), C::IDESC,
-                               (kb | j) != 0 ? 1u : 0u);
-                umma_commit(&empty[s]);  // the stage (A columns and B tile) is free once these finish
-            }
-            umma_commit(accfull);
-        }
-    } else {
-        // ------------------------------------------------------------ unpack into TMEM, then epilogue
-        const int q = warp & 3;            // TMEM lane quarter of this warp
-        const int r = 32 * q + lane;       // weight row within the tile (= TMEM lane)
-        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-        pdl_wait_prerequisites();
-        for (int i = threadIdx.x - 64; i < BT; i += 128) {
-            const int m = m0 + i;
-            fac[i] = m < M ? dequant_factor(*alpha, __ldg(scale_x + m), mode) : 0.0f;
-        }
-        const int sw = (r >> 2) & 1;  // 32B swizzle of the packed row
-        for (int kb = 0; kb < KB; ++kb) {
-            const int s = kb % C::STAGES;
-            if (kb >= C::STAGES && !mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1, status)) break;
-            if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, status)) break;
-            const uint32_t bp = smem_u32(smem + C::P_OFF + s * C::P_BYTES) + r * 32;
-            const uint4 p0 = lds128(bp + ((0 ^ sw) << 4));
-            const uint4 p1 = lds128(bp + ((1 ^ sw) << 4));
-            const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            uint32_t a[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint32_t s0 = w[c] & 0x33333333u;         // k = 16c + 0..7
-                const uint32_t s1 = (w[c] >> 2) & 0x33333333u;  // k = 16c + 8..15
-                a[4 * c + 0] = ternary4(s0);
-                a[4 * c + 1] = ternary4(s0 >> 16);
-                a[4 * c + 2] = ternary4(s1);
-                a[4 * c + 3] = ternary4(s1 >> 16);
-            }
-            tc_fence_after();  // order after the MMA that freed this stage
-            tmem_st_32x32b_x32(tmem_base + lane_off + C::A_COL0 + 32 * s, a);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&unpacked[s]);
-        }
-
-        // epilogue: TMEM lane r holds weight row n0 + r, column j token m0 + j
-        mbar_wait(accfull, 0, status);
-        tc_fence_after();
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four unpack warps: fac[] is complete
-        const int n = n0 + r;
-#pragma unroll 1
-        for (int c = 0; c < BT / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tmem_base + lane_off + 32 * c, v);
-            tmem_wait_ld();
-            if (n < N) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int m = m0 + 32 * c + j;
-                    if (m < M) {
-                        out[(int64_t)m * N + n] = __fmul_rn((float)(int)v[j], fac[32 * c + j]);
-                        if (acc_out) acc_out[(int64_t)m * N + n] = (int)v[j];
-                    }
+                if (wrapped && !mbar_wait_warp(SFREE + 8 * s, ph ^ 1u, status)) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx_elect(FULL + 8 * s, C::B_BYTES + C::P_BYTES);
+                tma_load_2d_elect(sP0 + s * C::P_BYTES, &tm_w, FULL + 8 * s, kb * (BK / 4), n0);
+                if (!waited) {
+                    pdl_wait_prerequisites();  // activation codes come from the previous kernel
+                    waited = true;
+                }
+                tma_load_2d_elect(sB0 + s * C::B_BYTES, &tm_act, FULL + 8 * s, kb * BK, m0);
+                if (++s == ST) {
+                    s = 0;
+                    ph ^= 1u;
+                    wrapped = true;
                 }
             }
         }
+        // every issued load must land before the CTA exits
+        for (int i = 0; i < ST; ++i) {
+            if (i < s) mbar_wait_warp(FULL + 8 * i, ph, status);
+            else if (wrapped) mbar_wait_warp(FULL + 8 * i, ph ^ 1u, status);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint64_t bdesc0 = smem_desc_sw128(sB0);
+        int s = 0, a = 0, tc = 0;
+        uint32_t ph = 0, aph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+            const int b = DB == 1 ? 0 : (tc & 1);
+            // the epilogue must have drained this buffer (its previous use was tile tc - DB)
+            if (tc >= DB && !mbar_wait_warp(ACCEMPTY + 8 * b, (uint32_t)((tc / DB) - 1) & 1u, status)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(b * BT);
+            for (int kb = 0; kb < KB; ++kb) {
+                if (!mbar_wait_warp(FULL + 8 * s, ph, status) || !mbar_wait_warp(UNPACKED + 8 * a, aph, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // the descriptor's start-address field advances by the stage offset / 16
+                const uint64_t bdesc = bdesc0 + (uint64_t)((uint32_t)(s * C::B_BYTES) >> 4);
+                const uint32_t a_tmem = tmem_base + C::A_COL0 + 32 * a;
+#pragma unroll
+                for (int j = 0; j < BK / 32; ++j)  // K = 32 per MMA: 8 TMEM columns of A, 32 bytes of B rows
+                    umma_i8_ts_elect(d_tmem, a_tmem + 8 * j, bdesc + (uint64_t)(2 * j), C::IDESC,
+                                     (kb | j) != 0 ? 1u : 0u);
+                umma_commit_elect(SFREE + 8 * s);  // stage s (activation tile, packed weights) is free
+                umma_commit_elect(AFREE + 8 * a);  // weight slot a is free
+                if (++s == ST) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                if (++a == AS) {
+                    a = 0;
+                    aph ^= 1u;
+                }
+            }
+            umma_commit_elect(ACCFULL + 8 * b);  // this tile's accumulator is complete
+        }
+    } else if (warp < 2 + 4 * UW) {
+        // ------------------------------------------------------------ unpack into TMEM
+        const int q = warp & 3;           // TMEM lane quarter of this warp
+        const int set = (warp - 2) >> 2;  // takes the stages it with it % UW == set
+        const int r = 32 * q + lane;      // weight row within the tile (= TMEM lane)
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        const uint32_t sw = (uint32_t)((r >> 2) & 1) << 4;  // 32B swizzle of the packed row
+        const uint32_t prow = sP0 + (uint32_t)r * 32;
+        int s = set, a = set, turn = 0;
+        uint32_t ph = 0, aph = 0;
+        bool awrapped = false, ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const bool mine = turn == set;
+                if (++turn == UW) turn = 0;
+                if (!mine) continue;
+                if (!mbar_wait_u32(FULL + 8 * s, ph, status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t bp = prow + s * C::P_BYTES;
+                const uint4 p0 = lds128(bp + (0u ^ sw));
+                const uint4 p1 = lds128(bp + (16u ^ sw));
+                const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                uint32_t av[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t s0 = w[c] & 0x33333333u;         // k = 16c + 0..7
+                    const uint32_t s1 = (w[c] >> 2) & 0x33333333u;  // k = 16c + 8..15
+                    av[4 * c + 0] = ternary4(s0);
+                    av[4 * c + 1] = ternary4(s0 >> 16);
+                    av[4 * c + 2] = ternary4(s1);
+                    av[4 * c + 3] = ternary4(s1 >> 16);
+                }
+                // the slot's previous use was stage it - AS
+                if (awrapped && !mbar_wait_u32(AFREE + 8 * a, aph ^ 1u, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();  // order after the MMA that freed this slot
+                tmem_st_32x32b_x32(tmem_base + lane_off + C::A_COL0 + 32 * a, av);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 2 * ST + a);
+                s += UW;
+                if (s >= ST) {
+                    s -= ST;
+                    ph ^= 1u;
+                }
+                a += UW;
+                if (a >= AS) {
+                    a -= AS;
+                    aph ^= 1u;
+                    awrapped = true;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int r = 32 * q + lane;  // weight row within the tile (= TMEM lane)
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        const int et = threadIdx.x - (64 + 128 * UW);  // 0..127
+        float *obuf = reinterpret_cast<float *>(smem + C::O_OFF);
+        const uint32_t sO0 = smem_u32(obuf);
+        if (et == 0 && tma_out) tma_prefetch_desc(&tm_out);
+        pdl_wait_prerequisites();
+        const float a_scale = *alpha;
+        int tc = 0, ck = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+            const int b = DB == 1 ? 0 : (tc & 1);
+            int n0, m0;
+            tmap.get(t, BT, n0, m0);
+            for (int i = et; i < BT; i += 128) {
+                const int m = m0 + i;
+                fac[b * BT + i] = m < M ? dequant_factor(a_scale, __ldg(scale_x + m), mode) : 0.0f;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (!mbar_wait_u32(ACCFULL + 8 * b, (uint32_t)(tc / DB) & 1u, status)) break;
+            tc_fence_after();
+            const int n = n0 + r;
+#pragma unroll 1
+            for (int c = 0; c < BT / 32; ++c) {
+                if (m0 + 32 * c >= M) break;  // the rest of the tile lies past the last token (uniform)
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_off + (uint32_t)(b * BT + 32 * c), v);
+                tmem_wait_ld();
+                if (tma_out) {
+                    // [32 tokens][128 rows] through shared memory, one bulk tensor store
+                    const int buf = ck & 1;
+                    if (et == 0 && ck >= 2) bulk_wait_group_read<1>();  // the store that read buf is done
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    float *sb = obuf + buf * (OUT_TOKENS * BW);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        sb[j * BW + r] = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                    fence_proxy_async_smem();
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (et == 0) {
+                        tma_store_2d(&tm_out, sO0 + (uint32_t)(buf * OUT_TOKENS * BW * 4), n0, m0 + 32 * c);
+                        bulk_commit_group();
+                    }
+                    ++ck;
+                } else if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + 32 * c + j;
+                        if (m < M) out[(int64_t)m * N + n] = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                    }
+                }
+                if (acc_out && n < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + 32 * c + j;
+                        if (m < M) acc_out[(int64_t)m * N + n] = (int)v[j];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + 2 * ST + 2 * AS + DB + b);  // the buffer may be overwritten
+            asm volatile("bar.sync 1, 128;" ::: "memory");              // fac row b is rewritten DB tiles later
+        }
+        if (et == 0 && tma_out) bulk_wait_group<0>();  // the last stores have landed
     }
 
     tc_fence_before();
@@ -249,16 +377,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
     }
 }
 
-template <int BT>
-cudaError_t launch_bt(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed, const float *alpha,
-                      int M, int N, int K, float *out, int32_t *acc_out, bool pdl, cudaStream_t s) {
-    using C = TcCfg<BT>;
-    CUtensorMap ta, tw;
-    if (!make_tmap_u8_2d(&ta, codes, (uint64_t)K, (uint64_t)M, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
+template <class C>
+cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
+                       const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
+                       cudaStream_t s) {
+    CUtensorMap ta, tw, to;
+    if (!make_tmap_u8_2d(&ta, codes, (uint64_t)K, (uint64_t)M, BK, C::BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!make_tmap_u8_2d(&tw, packed, (uint64_t)K / 4, (uint64_t)N, BK / 4, BW, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
-    auto kern = gemm_tc_kernel<BT>;
+    // The bulk-store epilogue needs a 16-byte row pitch and base, and a box that fits.
+    memset(&to, 0, sizeof(to));
+    const bool store_ok = N % 4 == 0 && M >= OUT_TOKENS && N >= BW && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+    const int tma_out = store_ok && make_tmap_f32_2d(&to, out, (uint64_t)N, (uint64_t)M, BW, OUT_TOKENS) ? 1 : 0;
+    auto kern = gemm_tc_kernel<C>;
     static bool done[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -268,9 +400,11 @@ cudaError_t launch_bt(const int8_t *codes, const float *scale_x, int mode, const
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) done[dev] = true;
     }
+    const long tiles = (long)((N + BW - 1) / BW) * ((M + C::BT - 1) / C::BT);
+    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + BW - 1) / BW), (unsigned)((M + BT - 1) / BT));
-    cfg.blockDim = dim3(THREADS);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr;
@@ -278,36 +412,60 @@ cudaError_t launch_bt(const int8_t *codes, const float *scale_x, int mode, const
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tw, scale_x, alpha, mode, M, N, K, out, acc_out, device_status_ptr());
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, scale_x, alpha, mode, M, N, K, out, acc_out,
+                              device_status_ptr());
 }
 
 }  // namespace
 
-// Relative cost of a token tile size: waves of CTAs times the per-tile work, over
-// the tile's efficiency (smaller tiles move more shared-memory bytes and unpack
-// more weights per MAC).
-double tile_cost(int BT, int M, int N, int sms) {
-    const double eff = BT >= 256 ? 1.0 : (BT >= 128 ? 0.85 : 0.65);
-    const int per_sm = BT <= 64 ? 2 : 1;
-    const long tiles = (long)((N + BW - 1) / BW) * ((M + BT - 1) / BT);
-    const long waves = (tiles + (long)sms * per_sm - 1) / ((long)sms * per_sm);
-    return (double)waves * BT / eff;
+// Modelled time of one token-tile size, in units of one 128-k stage of one tile:
+// rounds of tiles per SM x (stages per tile x relative stage cost + a drain stall
+// per tile when the accumulator is single-buffered).  The stage costs and the
+// stall are B200 measurements: a stage takes about as long at 192..256 tokens,
+// and the single-buffered 256-token tile stalls about 10 stages per tile.
+double gemm_tile_cost(int bt, int M, int N, int K, int sms) {
+    const double w = bt >= 192 ? 1.0 : (bt >= 128 ? 0.93 : 0.81);
+    const double drain = bt == 256 ? 10.0 : 0.0;
+    const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
+    const long rounds = (tiles + sms - 1) / sms;
+    return (double)rounds * ((double)(K / BK) * w + drain);
+}
+
+namespace {
+int g_forced_tile = 0;  // 0: automatic
+}  // namespace
+
+bool gemm_force_tile(int bt) {
+    if (bt != 0 && bt != 256 && bt != 224 && bt != 192 && bt != 128 && bt != 64) return false;
+    g_forced_tile = bt;
+    return true;
+}
+
+int gemm_pick_tile(int M, int N, int K, int sms) {
+    if (g_forced_tile) return g_forced_tile;
+    static const int cand[] = {224, 192, 128, 64};
+    int best = 256;
+    double best_cost = gemm_tile_cost(256, M, N, K, sms);
+    for (int bt : cand) {
+        const double c = gemm_tile_cost(bt, M, N, K, sms);
+        if (c < best_cost * 0.999) {
+            best = bt;
+            best_cost = c;
+        }
+    }
+    return best;
 }
 
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                            const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
                            cudaStream_t s) {
-    const int sms = sm_count();
-    int bt = 256;
-    double best = tile_cost(256, M, N, sms);
-    if (tile_cost(128, M, N, sms) < best) {
-        bt = 128;
-        best = tile_cost(128, M, N, sms);
+    switch (gemm_pick_tile(M, N, K, sm_count())) {
+    case 256: return launch_cfg<Cfg256>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
+    case 224: return launch_cfg<Cfg224>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
+    case 192: return launch_cfg<Cfg192>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
+    case 128: return launch_cfg<Cfg128>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
+    default: return launch_cfg<Cfg64>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
     }
-    if (M <= 64 && tile_cost(64, M, N, sms) < best) bt = 64;
-    if (bt == 256) return launch_bt<256>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    if (bt == 128) return launch_bt<128>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    return launch_bt<64>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
 }
 
 }  // namespace bitnet

@@ -17,6 +17,11 @@ constexpr int kGemvMaxM = 16;
 bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uint64_t rows,
                      uint32_t box_x, uint32_t box_y, CUtensorMapSwizzle swizzle);
 
+// 2D fp32 tensor map (no swizzle) over a row-major [rows][cols] array; cols * 4 and
+// the base must be 16-byte aligned.
+bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_x,
+                      uint32_t box_y);
+
 // Per-device address of the library's device status word.
 int *device_status_ptr();
 
@@ -30,7 +35,8 @@ size_t pack_workspace_bytes();
 cudaError_t launch_pack(const float *W, int64_t N, int64_t K, float eps, uint8_t *packed, float *alpha,
                         void *ws, cudaStream_t s);
 
-// Decode path (M <= 16): weight-streaming mma.sync kernel with cluster split-K.
+// Decode path (M <= 16): weight-streaming kernel, 2-bit weights unpacked in
+// registers, int8 mma.sync, split-K over the warps of one CTA.
 cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                         const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
                         bool pdl, cudaStream_t s);
@@ -39,6 +45,13 @@ cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, con
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                            const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
                            bool pdl, cudaStream_t s);
+
+// Token-tile size launch_gemm_tc uses for this shape on `sms` SMs (256/224/192/128/64,
+// or the forced value), and the modelled cost the automatic choice compares.
+int gemm_pick_tile(int M, int N, int K, int sms);
+double gemm_tile_cost(int bt, int M, int N, int K, int sms);
+// Force the token tile (0 = automatic); false for an unsupported value.
+bool gemm_force_tile(int bt);
 
 // Launch the timeout self-test kernel.
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);

@@ -27,10 +27,27 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 1
+    assert L.bitnet_abi_version() == 2
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
+
+
+def test_gemm_token_tile_host_logic(L):
+    # decode-sized and rejected problems are answered on the host, without touching a GPU
+    assert L.bitnet_gemm_token_tile(16, 4096, 4096) == 0
+    assert L.bitnet_gemm_token_tile(1, 2560, 6912) == 0
+    assert L.bitnet_gemm_token_tile(-1, 256, 256) == -1
+    assert L.bitnet_gemm_token_tile(64, 0, 256) == -1
+    assert L.bitnet_gemm_token_tile(64, 256, 100) == -1
+    for bad in (1, 32, 96, 160, 255, 257, 512, -64):
+        assert L.bitnet_gemm_force_token_tile(bad) == _native.ERR_INVALID_ARG
+    try:
+        for good in (256, 224, 192, 128, 64):
+            assert L.bitnet_gemm_force_token_tile(good) == _native.OK
+            assert L.bitnet_gemm_token_tile(4096, 4096, 4096) == good  # a forced tile wins
+    finally:
+        assert L.bitnet_gemm_force_token_tile(0) == _native.OK
 
 
 def test_workspace_sizes(L):

@@ -129,9 +129,9 @@ GEMM_SHAPES = [
     # decode kernel (M <= 16)
     (1, 64, 128), (2, 100, 384), (5, 700, 2560), (8, 6912, 2560), (8, 2560, 6912), (9, 130, 640),
     (16, 512, 1024),
-    # tcgen05 kernel
+    # tcgen05 kernel with its automatic token tile (few tiles: small tiles spread over the SMs)
     (17, 256, 128), (64, 200, 640), (128, 256, 256), (130, 300, 384), (256, 520, 1024), (300, 1000, 2048),
-    (1200, 2560, 128),  # large enough for the 256-token tile
+    (1200, 2560, 128), (2048, 2560, 256), (2000, 2600, 384), (1051, 4096, 256), (64, 40000, 128),
 ]
 
 
@@ -151,6 +151,39 @@ def test_gemm_exact_accumulators(M, N, K, mode):
     np.testing.assert_array_equal(host(acc), acc_ref)
     out_ref = ref.dequant(acc_ref, scale, alpha[0], MODES[mode])
     np.testing.assert_array_equal(host(out), out_ref)
+
+
+def _gemm_case(M, N, K, mode, seed):
+    rng = np.random.default_rng(seed)
+    lo, hi = (-128, 128) if mode == "int8" else (-8, 8)
+    q = rng.integers(lo, hi, size=(M, K)).astype(np.int8)
+    t = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    return q, ref.pack(t), rng.uniform(0.1, 10.0, size=M).astype(np.float32), np.array([0.0173], np.float32)
+
+
+@pytest.mark.parametrize("tile", [256, 224, 192, 128, 64])
+def test_gemm_forced_token_tiles(tile):
+    # Every token-tile configuration of the tcgen05 kernel, forced, on: several rounds of
+    # tiles per SM with ragged tokens and weight rows (bulk-store epilogue); N % 4 != 0 and
+    # M < 32 (direct-store epilogue).  Accumulators and outputs must be exact.
+    cases = [(10 * tile + 37, 1988, 128), (77, 130, 384), (20, 256, 256)]
+    try:
+        tb.bitnet_gemm_force_token_tile(tile)
+        for i, (M, N, K) in enumerate(cases):
+            assert tb.bitnet_gemm_token_tile(M, N, K) == tile
+            mode = ("int8", "int4")[i % 2]
+            q, packed, scale, alpha = _gemm_case(M, N, K, mode, seed=tile * 10 + i)
+            acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+            out = tb.bitnet_ternary_gemm(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, acc_out=acc)
+            out2 = tb.bitnet_ternary_gemm(dev(q), dev(scale), mode, dev(packed), dev(alpha), N)
+            acc_ref = ref.gemm_packed(q, packed, N)
+            np.testing.assert_array_equal(host(acc), acc_ref, err_msg=f"tile {tile} {M}x{N}x{K}")
+            out_ref = ref.dequant(acc_ref, scale, alpha[0], MODES[mode])
+            np.testing.assert_array_equal(host(out), out_ref)
+            np.testing.assert_array_equal(host(out2), out_ref)
+        assert tb.bitnet_get_last_device_status() == 0
+    finally:
+        tb.bitnet_gemm_force_token_tile(0)
 
 
 def test_gemm_extreme_codes():
