@@ -18,7 +18,17 @@
  *     only a per-device cache of kernel attributes and one 4-byte device status word.
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call only enqueues work on that stream and returns without
- *     synchronising; results are ready when the stream reaches them.
+ *     synchronising; results are ready when the stream reaches them.  The kernels
+ *     use programmatic dependent launch: they may begin while the previous kernel on
+ *     the stream finishes.  Before their dependency wait they read only the packed
+ *     weights (prefetch and first loads); every other input is read after it.  So
+ *     `packed` must not be written by the kernel immediately preceding a call on its
+ *     stream, unless that kernel is bitnet_pack_ternary's (it fences its stores) or
+ *     ends every writing thread with __threadfence(); copies, events, other streams
+ *     and anything earlier are unaffected.  A following kernel launched with
+ *     programmatic dependent launch must itself wait (cudaGridDependencySynchronize)
+ *     before reading a call's outputs; kernels launched without it start after the
+ *     call completes, as usual.
  *   - Errors: every call validates its arguments on the host before launching
  *     anything and returns a bitnet_status_t; nothing throws or aborts.  A kernel
  *     that gives up on a bounded wait records BITNET_ERR_TIMEOUT in the device

@@ -187,9 +187,11 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
     extern __shared__ __align__(16) float sm[];  // K + K/32 floats (padded)
     __shared__ float red[32];
 
-    // X may come from the previous kernel: wait for it, then let the GEMM start streaming weights.
-    pdl_wait_prerequisites();
+    // Let the GEMM launch now and start streaming its weights; then wait for X, which
+    // may come from the previous kernel.  The GEMM waits for this kernel before it
+    // reads the codes, so the order of the data is kept.
     pdl_launch_dependents();
+    pdl_wait_prerequisites();
 
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
@@ -300,8 +302,8 @@ __global__ void __launch_bounds__(T)
 act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gain, int K, float eps,
                        int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x) {
     __shared__ float red[32];
+    pdl_launch_dependents();  // as in the FWHT kernel: the GEMM may launch, X is waited for
     pdl_wait_prerequisites();
-    pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
     const int K4 = K >> 2;
@@ -358,8 +360,9 @@ act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gai
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while the
-// previous kernel of the stream finishes; it waits (griddepcontrol.wait) before
-// reading anything, and only then lets its own dependents start.
+// previous kernel of the stream finishes.  It lets its own dependents launch at once
+// and waits (griddepcontrol.wait) before reading anything; the dependents in turn
+// only prefetch weights into L2 before their own wait.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
     cudaLaunchConfig_t cfg = {};

@@ -211,7 +211,7 @@ bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x, b
                                     float *out, int32_t *acc_out, void *stream) {
     bitnet_status_t st = validate_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out);
     if (st != BITNET_OK || M == 0) return st;
-    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, false,
+    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, true,
                               static_cast<cudaStream_t>(stream)));
 }
 

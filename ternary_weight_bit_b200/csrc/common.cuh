@@ -152,6 +152,16 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- L2 prefetch
+// Bulk prefetch of [src, src + bytes) into L2 (src 16-byte aligned, bytes a multiple
+// of 16).  Kernels issue it before their dependency wait: a prefetch cannot expose
+// data that a preceding kernel is still writing (L2 is the point of coherence), and
+// the real loads after the wait then hit L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- bulk stores
 // 2D tiled TMA store shared -> global (bulk-group completion).  x * elem_size must
 // be a multiple of 16 and no coordinate may be negative; parts of the box beyond

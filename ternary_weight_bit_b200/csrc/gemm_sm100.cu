@@ -124,7 +124,8 @@ struct TileMap {
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w,
-               const __grid_constant__ CUtensorMap tm_out, int tma_out, const float *__restrict__ scale_x,
+               const __grid_constant__ CUtensorMap tm_out, int tma_out, const uint8_t *__restrict__ packed,
+               const float *__restrict__ scale_x,
                const float *__restrict__ alpha, int mode, int M, int N, int K, float *__restrict__ out,
                int32_t *__restrict__ acc_out, int *status) {
     constexpr int BT = C::BT, ST = C::ST, AS = C::AS, DB = C::DB, UW = C::UW;
@@ -173,8 +174,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
             tma_prefetch_desc(&tm_act);
             tma_prefetch_desc(&tm_w);
         }
+        // Before the dependency wait only an L2 prefetch of the first tile's weight rows
+        // (contiguous: 128 rows x K/4 bytes, at most 128 KB) is issued; every TMA load
+        // follows the wait.
+        if (lane == 0 && (int)blockIdx.x < tiles) {
+            int n0, m0;
+            tmap.get(blockIdx.x, BT, n0, m0);
+            const int nrows = (N - n0) < BW ? (N - n0) : BW;
+            const uint32_t bytes = (uint32_t)nrows * (uint32_t)(K / 4);
+            bulk_prefetch_l2(packed + (int64_t)n0 * (K / 4), bytes < (128u << 10) ? bytes : (128u << 10));
+        }
         __syncwarp();
-        bool waited = false, ok = true, wrapped = false;
+        pdl_launch_dependents();   // the next kernel may launch; it waits for this grid
+        pdl_wait_prerequisites();  // activation codes come from the previous kernel
+        bool ok = true, wrapped = false;
         int s = 0;
         uint32_t ph = 0;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
@@ -187,10 +200,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
                 }
                 mbar_expect_tx_elect(FULL + 8 * s, C::B_BYTES + C::P_BYTES);
                 tma_load_2d_elect(sP0 + s * C::P_BYTES, &tm_w, FULL + 8 * s, kb * (BK / 4), n0);
-                if (!waited) {
-                    pdl_wait_prerequisites();  // activation codes come from the previous kernel
-                    waited = true;
-                }
                 tma_load_2d_elect(sB0 + s * C::B_BYTES, &tm_act, FULL + 8 * s, kb * BK, m0);
                 if (++s == ST) {
                     s = 0;
@@ -412,7 +421,7 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, scale_x, alpha, mode, M, N, K, out, acc_out,
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, packed, scale_x, alpha, mode, M, N, K, out, acc_out,
                               device_status_ptr());
 }
 

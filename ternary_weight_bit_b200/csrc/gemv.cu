@@ -16,9 +16,10 @@
 // (8 per chunk) takes packed word s/2, half s%2 (weights: one mask, one shift and two
 // byte permutes per row) and activation bytes 8s..8s+7.  Weights go on the 16-row A
 // side of mma.sync m16n8k32 s8, tokens on the 8-column B side.  Each warp keeps up to
-// PF chunks of loads in flight; the weight loads of its first chunks are issued before
-// griddepcontrol.wait, so with programmatic dependent launch they overlap the
-// activation-quantisation kernel.
+// PF chunks of loads in flight.  Launched with programmatic dependent launch, a CTA
+// loads its first chunks and bulk-prefetches the rest of its 16 weight rows into L2
+// before the dependency wait, so the weight stream overlaps the kernels before it;
+// every kernel of the path triggers its dependents at its start.
 #include "common.cuh"
 #include "host.h"
 
@@ -66,8 +67,15 @@ gemv_kernel(const uint8_t *__restrict__ packed, const int8_t *__restrict__ codes
     const uint8_t *wrow0 = packed + (int64_t)(v0 ? n0 + g : 0) * rb + 16 * t;
     const uint8_t *wrow1 = packed + (int64_t)(v1 ? n0 + g + 8 : 0) * rb + 16 * t;
 
+    // Weights do not depend on the previous kernel (see the stream contract in
+    // bitnet.h): before the dependency wait, load the first PF chunks of every warp
+    // into registers and bulk-prefetch the rest of each of the CTA's 16 rows into L2.
+    {
+        const int64_t pre = (int64_t)PF * WK * 64;  // bytes of each row the first loads cover
+        if (pre < rb && threadIdx.x < ROWS && n0 + (int)threadIdx.x < N)
+            bulk_prefetch_l2(packed + (int64_t)(n0 + threadIdx.x) * rb + pre, (uint32_t)(rb - pre));
+    }
     Chunk<NT> buf[PF];
-    // weights of the first chunks: independent of the previous kernel
 #pragma unroll
     for (int j = 0; j < PF; ++j) {
         const int c = warp + j * WK;
@@ -75,7 +83,10 @@ gemv_kernel(const uint8_t *__restrict__ packed, const int8_t *__restrict__ codes
         buf[j].w0 = (in && v0) ? ldg_stream(wrow0 + 64 * c) : make_uint4(0, 0, 0, 0);
         buf[j].w1 = (in && v1) ? ldg_stream(wrow1 + 64 * c) : make_uint4(0, 0, 0, 0);
     }
-    pdl_wait_prerequisites();  // codes and scales come from the previous kernel
+    // The next kernel of the stream may launch now (it waits for this grid before
+    // reading anything this grid writes); then wait for the codes and scales.
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();
     if (threadIdx.x < TOK)
         fac[threadIdx.x] = (int)threadIdx.x < M ? dequant_factor(*alpha, __ldg(scale_x + threadIdx.x), mode) : 0.0f;
 

@@ -84,6 +84,10 @@ pack_words(const float *__restrict__ W, int64_t words, float eps, const float *_
         out |= code << (4 * i + 2 * h);
     }
     packed[w] = out;
+    // The GEMV/GEMM kernels of a following forward may load packed weights before their
+    // programmatic-launch dependency wait (they can launch as soon as this grid exits).
+    // The fence makes this thread's store visible device-wide before the grid exits.
+    __threadfence();
 }
 
 }  // namespace
