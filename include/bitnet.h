@@ -157,7 +157,9 @@ BITNET_API bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float 
  * Definition: bitnet_v2_engine.py page, HBitLinear.forward, Eq. 7.
  *   Arguments as in the two calls above; ws is device scratch of at least
  *   bitnet_forward_workspace_bytes(M, K) bytes holding the int8 codes and the
- *   per-token scales between the two kernels (BITNET_ERR_WORKSPACE if smaller).
+ *   per-token scales between the two kernels, and 4 KB of tile counters for a
+ *   split-K GEMM (BITNET_ERR_WORKSPACE if smaller).  Its contents need no
+ *   initialisation.
  * ------------------------------------------------------------------------ */
 BITNET_API size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K);
 BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M,
@@ -178,7 +180,7 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype
  *   BITNET_NOALLOC_SCRATCH_BYTES in the library's own device memory; every GPU that
  *   loads the library holds that array until the process exits.  A call needs
  *   bitnet_forward_workspace_bytes(M, K) <= BITNET_NOALLOC_SCRATCH_BYTES (4 MiB:
- *   for example M*K up to about 4.19 million); larger calls return
+ *   for example M*K up to about 4.18 million); larger calls return
  *   BITNET_ERR_WORKSPACE without launching anything.
  *   The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  *   routine).  Its first call on a device looks up the array's device address
@@ -199,9 +201,16 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
 /* --------------------------------------------------------------------------
  * Prefill GEMM tile control (no counterpart on the pages).
  * bitnet_gemm_token_tile: the token-tile size (256, 224, 192, 128 or 64 tokens
- *   per tensor-core tile) that bitnet_ternary_gemm and the forwards use for an
- *   M x N x K problem on the current device; 0 when M <= 16 (the decode kernel
- *   runs instead); -1 for sizes the GEMM rejects.  Includes any forced value.
+ *   per tensor-core tile) that bitnet_ternary_gemm uses for an M x N x K problem
+ *   on the current device; 0 when M <= 16 (the decode kernel runs instead); -1 for
+ *   sizes the GEMM rejects.  Includes any forced value.
+ * bitnet_forward_gemm_plan: the plan of the GEMM inside bitnet_hbitlinear_forward
+ *   (and _noalloc) for the same problem: returns the token tile as above and writes
+ *   the k-split count to *k_splits (if not NULL).  When the output has few tiles
+ *   for the SMs, the forward splits K over up to 8 CTAs per tile: the partial int32
+ *   sums are added with integer atomics (exact, order-independent) into `out`,
+ *   which act_quant zeroes first, and the last split of each tile dequantises in
+ *   place.  The result is bit-identical to the unsplit GEMM on the same codes.
  * bitnet_gemm_force_token_tile: process-wide override of that choice, for every
  *   device and thread: 0 restores the automatic choice; 256, 224, 192, 128 or 64
  *   forces it; any other value returns BITNET_ERR_INVALID_ARG and changes nothing.
@@ -210,6 +219,7 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
  *   while no other thread is launching GEMMs.
  * ------------------------------------------------------------------------ */
 BITNET_API int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K);
+BITNET_API int bitnet_forward_gemm_plan(int64_t M, int64_t N, int64_t K, int *k_splits);
 BITNET_API bitnet_status_t bitnet_gemm_force_token_tile(int token_tile);
 
 /* --------------------------------------------------------------------------

@@ -25,7 +25,7 @@ __all__ = [
     "BitnetError", "HBitLinear", "bitnet_pack_ternary", "bitnet_act_quant", "bitnet_ternary_gemm",
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
-    "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile",
+    "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_forward_gemm_plan",
 ]
 
 _MODES = {"int8": _native.ACT_INT8_ABSMAX, "int4": _native.ACT_INT4_ABSMEAN}
@@ -69,6 +69,13 @@ def bitnet_abi_version() -> int:
 def bitnet_gemm_token_tile(M: int, N: int, K: int) -> int:
     """Token-tile size of the tcgen05 GEMM for this shape (0: decode kernel, -1: rejected)."""
     return _native.load().bitnet_gemm_token_tile(M, N, K)
+
+
+def bitnet_forward_gemm_plan(M: int, N: int, K: int) -> tuple:
+    """(token tile, k-splits) of the GEMM inside the forward; (0, 0) for the decode kernel."""
+    sp = ctypes.c_int(0)
+    tile = _native.load().bitnet_forward_gemm_plan(M, N, K, ctypes.byref(sp))
+    return tile, sp.value
 
 
 def bitnet_gemm_force_token_tile(token_tile: int) -> None:

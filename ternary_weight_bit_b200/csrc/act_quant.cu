@@ -17,6 +17,7 @@
 // (exact for even LOGK).  This reorders the roundings of the page's per-stage
 // scaling; results differ from it only in the last bits.
 #include "common.cuh"
+#include "host.h"
 
 namespace bitnet {
 
@@ -178,10 +179,21 @@ __device__ __forceinline__ int reg_part(int p, int r) {
 // compile-time offset from one per-thread base.
 __device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
 
+// Zero the token's row of a following split-K GEMM's output (it adds int32 partial
+// sums there) and, in CTA 0, that GEMM's tile counters.  Runs after the dependency
+// wait: the buffers may still be read by earlier kernels until then.
+__device__ __forceinline__ void zero_fill(const ZeroFill &z) {
+    if (!z.rows) return;
+    uint32_t *row = z.rows + (int64_t)blockIdx.x * z.row_words;
+    for (int i = threadIdx.x; i < z.row_words; i += blockDim.x) row[i] = 0u;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < z.cnt_n; i += blockDim.x) z.cnt[i] = 0;
+}
+
 template <int LOGK, bool BF16>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::T)
 act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain, float eps, int mode,
-                      int8_t *__restrict__ codes, float *__restrict__ scale_x) {
+                      int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
     using S = FwhtShape<LOGK>;
     constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
     extern __shared__ __align__(16) float sm[];  // K + K/32 floats (padded)
@@ -192,6 +204,7 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
     // reads the codes, so the order of the data is kept.
     pdl_launch_dependents();
     pdl_wait_prerequisites();
+    zero_fill(zf);
 
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
@@ -300,10 +313,11 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
 template <int T, int NV, bool BF16>
 __global__ void __launch_bounds__(T)
 act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gain, int K, float eps,
-                       int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x) {
+                       int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
     __shared__ float red[32];
     pdl_launch_dependents();  // as in the FWHT kernel: the GEMM may launch, X is waited for
     pdl_wait_prerequisites();
+    zero_fill(zf);
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
     const int K4 = K >> 2;
@@ -380,7 +394,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 template <int LOGK, bool BF16>
 cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
-                        float *scale_x, cudaStream_t s) {
+                        float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     using S = FwhtShape<LOGK>;
     const size_t smem = (size_t)(S::K + S::K / 32) * sizeof(float);
     auto kern = act_quant_fwht_kernel<LOGK, BF16>;
@@ -395,41 +409,41 @@ cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, 
             if (dev < kMaxDevices) done[dev] = true;
         }
     }
-    return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, X, gain, eps, mode, codes, scale_x);
+    return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, X, gain, eps, mode, codes, scale_x, zf);
 }
 
 template <int NV, bool BF16>
 cudaError_t launch_plain(const void *X, int64_t M, int K, const float *gain, float eps, int mode,
-                         int8_t *codes, float *scale_x, cudaStream_t s) {
+                         int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     constexpr int T = 256;
     return launch_pdl(act_quant_plain_kernel<T, NV, BF16>, dim3((unsigned)M), dim3(T), 0, s, X, gain, K, eps, mode,
-                      codes, scale_x);
+                      codes, scale_x, zf);
 }
 
 template <bool BF16>
 cudaError_t dispatch(const void *X, int64_t M, int K, const float *gain, float eps, int fwht, int mode,
-                     int8_t *codes, float *scale_x, cudaStream_t s) {
+                     int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     if (fwht) {
         switch (__builtin_ctz((unsigned)K)) {
-            case 7: return launch_fwht<7, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 8: return launch_fwht<8, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 9: return launch_fwht<9, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 10: return launch_fwht<10, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 11: return launch_fwht<11, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 12: return launch_fwht<12, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 13: return launch_fwht<13, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 14: return launch_fwht<14, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
-            case 15: return launch_fwht<15, BF16>(X, M, gain, eps, mode, codes, scale_x, s);
+            case 7: return launch_fwht<7, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 8: return launch_fwht<8, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 9: return launch_fwht<9, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 10: return launch_fwht<10, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 11: return launch_fwht<11, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 12: return launch_fwht<12, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 13: return launch_fwht<13, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 14: return launch_fwht<14, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 15: return launch_fwht<15, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
             default: return cudaErrorInvalidValue;
         }
     }
     const int nv = (int)ceil_div(K / 4, 256);
-    if (nv <= 1) return launch_plain<1, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
-    if (nv <= 2) return launch_plain<2, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
-    if (nv <= 4) return launch_plain<4, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
-    if (nv <= 8) return launch_plain<8, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
-    if (nv <= 16) return launch_plain<16, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
-    if (nv <= 32) return launch_plain<32, BF16>(X, M, K, gain, eps, mode, codes, scale_x, s);
+    if (nv <= 1) return launch_plain<1, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 2) return launch_plain<2, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 4) return launch_plain<4, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 8) return launch_plain<8, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 16) return launch_plain<16, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 32) return launch_plain<32, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
     return cudaErrorInvalidValue;
 }
 
@@ -437,10 +451,10 @@ cudaError_t dispatch(const void *X, int64_t M, int K, const float *gain, float e
 
 // Host entry used by the ABI layer (arguments already validated).
 cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
-                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s) {
+                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s, ZeroFill zf) {
     if (M == 0) return cudaSuccess;
-    return bf16 ? dispatch<true>(X, M, K, gain, eps, fwht, mode, codes, scale_x, s)
-                : dispatch<false>(X, M, K, gain, eps, fwht, mode, codes, scale_x, s);
+    return bf16 ? dispatch<true>(X, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s)
+                : dispatch<false>(X, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s);
 }
 
 }  // namespace bitnet

@@ -153,6 +153,31 @@ cudaError_t run_gemm(const int8_t *codes, const float *scale_x, int mode, const 
 
 }  // namespace
 
+// act_quant into (codes, scale_x), then the GEMV or the tcgen05 GEMM, the second
+// launched with programmatic dependent launch.  A GEMM whose output has few tiles
+// splits K: act_quant then also zeroes `out` and the tile counters for it.
+cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
+                            int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
+                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s) {
+    GemmPlan plan{0, 1};
+    ZeroFill zf;
+    if (M > kGemvMaxM) {
+        plan = gemm_plan((int)M, (int)N, (int)K, sm_count(), kSplitCounters);
+        if (plan.splits > 1) {
+            zf.rows = reinterpret_cast<uint32_t *>(out);
+            zf.row_words = (int)N;
+            zf.cnt = tile_cnt;
+            zf.cnt_n = (int)(((N + 127) / 128) * ((M + plan.token_tile - 1) / plan.token_tile));
+        }
+    }
+    cudaError_t e = launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s, zf);
+    if (e != cudaSuccess) return e;
+    if (M <= kGemvMaxM)
+        return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s);
+    return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s, plan,
+                          tile_cnt);
+}
+
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s) {
     wait_selftest_kernel<<<1, 32, 0, s>>>((uint64_t)limit_us * 1000ull, device_status_ptr());
     return cudaGetLastError();
@@ -216,8 +241,10 @@ bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x, b
 }
 
 size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K) {
-    if (M < 0 || K < 0) return 0;
-    return align256((size_t)M * (size_t)K) + align256((size_t)M * sizeof(float));
+    if (M <= 0 || K < 0) return 0;
+    // codes [M][K], scales [M], then the split-K tile counters of the GEMM
+    return align256((size_t)M * (size_t)K) + align256((size_t)M * sizeof(float)) +
+           (size_t)kSplitCounters * sizeof(int);
 }
 
 bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
@@ -233,16 +260,24 @@ bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int
         return BITNET_ERR_WORKSPACE;
     int8_t *codes = static_cast<int8_t *>(ws);
     float *scale_x = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)M * (size_t)K));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s);
-    if (e != cudaSuccess) return BITNET_ERR_CUDA;
-    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, nullptr, true, s));
+    int *tile_cnt = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(scale_x) + align256((size_t)M * sizeof(float)));
+    return from_cuda(forward_kernels(X, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, codes, scale_x,
+                                     tile_cnt, static_cast<cudaStream_t>(stream)));
 }
 
 int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {
     if (M < 0 || N < 1 || N > kMaxRows || check_k(K, 0) != BITNET_OK) return -1;
     if (M <= kGemvMaxM) return 0;
     return gemm_pick_tile((int)M, (int)N, (int)K, sm_count());
+}
+
+int bitnet_forward_gemm_plan(int64_t M, int64_t N, int64_t K, int *k_splits) {
+    if (k_splits) *k_splits = 0;
+    if (M < 0 || N < 1 || N > kMaxRows || check_k(K, 0) != BITNET_OK) return -1;
+    if (M <= kGemvMaxM) return 0;
+    const GemmPlan p = gemm_plan((int)M, (int)N, (int)K, sm_count(), kSplitCounters);
+    if (k_splits) *k_splits = p.splits;
+    return p.token_tile;
 }
 
 bitnet_status_t bitnet_gemm_force_token_tile(int token_tile) {

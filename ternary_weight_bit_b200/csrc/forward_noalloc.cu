@@ -72,22 +72,21 @@ extern "C" bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
     if (!X || !packed || !alpha || !out) return BITNET_ERR_INVALID_ARG;
     if (!aligned16(X) || !aligned16(packed) || !aligned16(alpha) || !aligned16(out) || (gain && !aligned16(gain)))
         return BITNET_ERR_INVALID_ARG;
-    // Codes [M][K] then scales [M], each 256-byte aligned, must fit the fixed array.
+    // Codes [M][K], scales [M] (each 256-byte aligned) and the split-K tile counters
+    // must fit the fixed array.
     const size_t codes_bytes = round256((size_t)M * (size_t)K);
-    const size_t need = codes_bytes + round256((size_t)M * sizeof(float));
+    const size_t scales_bytes = round256((size_t)M * sizeof(float));
+    const size_t need = codes_bytes + scales_bytes + (size_t)kSplitCounters * sizeof(int);
     if (need > kNoAllocScratchBytes) return BITNET_ERR_WORKSPACE;
 
     uint8_t *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return BITNET_ERR_CUDA;
     int8_t *codes = reinterpret_cast<int8_t *>(scratch);
     float *scale_x = reinterpret_cast<float *>(scratch + codes_bytes);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // Nothing in the array needs clearing: act_quant writes every code and scale the GEMM reads.
-    if (launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s) != cudaSuccess)
-        return BITNET_ERR_CUDA;
-    cudaError_t e = M <= kGemvMaxM
-                        ? launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s)
-                        : launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr,
-                                         true, s);
+    int *tile_cnt = reinterpret_cast<int *>(scratch + codes_bytes + scales_bytes);
+    // Nothing in the array needs clearing beforehand: act_quant writes every code and
+    // scale the GEMM reads, and zeroes the counters when the GEMM splits K.
+    const cudaError_t e = forward_kernels(X, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, codes, scale_x,
+                                          tile_cnt, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }

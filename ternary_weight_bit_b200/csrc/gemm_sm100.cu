@@ -127,7 +127,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
                const __grid_constant__ CUtensorMap tm_out, int tma_out, const uint8_t *__restrict__ packed,
                const float *__restrict__ scale_x,
                const float *__restrict__ alpha, int mode, int M, int N, int K, float *__restrict__ out,
-               int32_t *__restrict__ acc_out, int *status) {
+               int32_t *__restrict__ acc_out, int splits, int *__restrict__ tile_cnt, int *status) {
     constexpr int BT = C::BT, ST = C::ST, AS = C::AS, DB = C::DB, UW = C::UW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,12 +137,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
                    AFREE = UNPACKED + 8 * AS, ACCFULL = AFREE + 8 * AS, ACCEMPTY = ACCFULL + 8 * DB;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::TMEM_SLOT_OFF);
     float *fac = reinterpret_cast<float *>(smem + C::F_OFF);
+    __shared__ int s_last;  // split-K: this CTA added the last split of the tile
     const uint32_t sB0 = smem_u32(smem + C::B_OFF), sP0 = smem_u32(smem + C::P_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB = K / BK;
+    // Work unit u = (output tile u / splits, k-split u % splits); a split covers KBS
+    // consecutive 128-k stages (splits divides K / 128).
+    const int KBS = K / BK / splits;
     const TileMap tmap{(N + BW - 1) / BW};
     const int tiles = tmap.nb_blocks * ((M + BT - 1) / BT);
+    const int units = tiles * splits;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < ST; ++i) {
@@ -177,9 +181,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         // Before the dependency wait only an L2 prefetch of the first tile's weight rows
         // (contiguous: 128 rows x K/4 bytes, at most 128 KB) is issued; every TMA load
         // follows the wait.
-        if (lane == 0 && (int)blockIdx.x < tiles) {
+        if (lane == 0 && (int)blockIdx.x < units) {
             int n0, m0;
-            tmap.get(blockIdx.x, BT, n0, m0);
+            tmap.get((int)blockIdx.x / splits, BT, n0, m0);
             const int nrows = (N - n0) < BW ? (N - n0) : BW;
             const uint32_t bytes = (uint32_t)nrows * (uint32_t)(K / 4);
             bulk_prefetch_l2(packed + (int64_t)n0 * (K / 4), bytes < (128u << 10) ? bytes : (128u << 10));
@@ -190,10 +194,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         bool ok = true, wrapped = false;
         int s = 0;
         uint32_t ph = 0;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int n0, m0;
-            tmap.get(t, BT, n0, m0);
-            for (int kb = 0; kb < KB; ++kb) {
+            tmap.get(u / splits, BT, n0, m0);
+            const int kb0 = (u % splits) * KBS;
+            for (int kb = kb0; kb < kb0 + KBS; ++kb) {
                 if (wrapped && !mbar_wait_warp(SFREE + 8 * s, ph ^ 1u, status)) {
                     ok = false;
                     break;
@@ -219,13 +224,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         int s = 0, a = 0, tc = 0;
         uint32_t ph = 0, aph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tc) {
             const int b = DB == 1 ? 0 : (tc & 1);
-            // the epilogue must have drained this buffer (its previous use was tile tc - DB)
+            // the epilogue must have drained this buffer (its previous use was unit tc - DB)
             if (tc >= DB && !mbar_wait_warp(ACCEMPTY + 8 * b, (uint32_t)((tc / DB) - 1) & 1u, status)) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(b * BT);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < KBS; ++kb) {
                 if (!mbar_wait_warp(FULL + 8 * s, ph, status) || !mbar_wait_warp(UNPACKED + 8 * a, aph, status)) {
                     ok = false;
                     break;
@@ -262,8 +267,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         int s = set, a = set, turn = 0;
         uint32_t ph = 0, aph = 0;
         bool awrapped = false, ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            for (int kb = 0; kb < KB; ++kb) {
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int kb = 0; kb < KBS; ++kb) {
                 const bool mine = turn == set;
                 if (++turn == UW) turn = 0;
                 if (!mine) continue;
@@ -321,10 +326,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         pdl_wait_prerequisites();
         const float a_scale = *alpha;
         int tc = 0, ck = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+        int32_t *acc_img = reinterpret_cast<int32_t *>(out);  // split-K: out holds int32 sums first
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++tc) {
             const int b = DB == 1 ? 0 : (tc & 1);
+            const int tile = u / splits;
             int n0, m0;
-            tmap.get(t, BT, n0, m0);
+            tmap.get(tile, BT, n0, m0);
             for (int i = et; i < BT; i += 128) {
                 const int m = m0 + i;
                 fac[b * BT + i] = m < M ? dequant_factor(a_scale, __ldg(scale_x + m), mode) : 0.0f;
@@ -333,6 +340,56 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
             if (!mbar_wait_u32(ACCFULL + 8 * b, (uint32_t)(tc / DB) & 1u, status)) break;
             tc_fence_after();
             const int n = n0 + r;
+            if (splits > 1) {
+                // Add this split's partial sums to the int32 image of the tile (integer
+                // atomics: the total does not depend on their order).
+#pragma unroll 1
+                for (int c = 0; c < BT / 32; ++c) {
+                    if (m0 + 32 * c >= M) break;
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem_base + lane_off + (uint32_t)(b * BT + 32 * c), v);
+                    tmem_wait_ld();
+                    if (n < N) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int m = m0 + 32 * c + j;
+                            if (m < M) atomicAdd(acc_img + (int64_t)m * N + n, (int)v[j]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 2 * ST + 2 * AS + DB + b);  // the buffer may be overwritten
+                __threadfence();  // this thread's additions are performed before the count below
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (et == 0) s_last = atomicAdd(tile_cnt + tile, 1) == splits - 1;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (s_last) {
+                    // the last split of this tile: dequantise the sums in place
+                    __threadfence();
+#pragma unroll 1
+                    for (int c = 0; c < BT / 32; ++c) {
+                        if (m0 + 32 * c >= M || n >= N) break;
+                        int32_t sums[32];  // all 32 loads in flight before any use
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int m = m0 + 32 * c + j;
+                            sums[j] = m < M ? __ldcg(acc_img + (int64_t)m * N + n) : 0;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int m = m0 + 32 * c + j;
+                            if (m < M) {
+                                out[(int64_t)m * N + n] = __fmul_rn((float)sums[j], fac[b * BT + 32 * c + j]);
+                                if (acc_out) acc_out[(int64_t)m * N + n] = sums[j];
+                            }
+                        }
+                    }
+                    if (et == 0) tile_cnt[tile] = 0;  // ready for the next call
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // fac row b and s_last are reused
+                continue;
+            }
 #pragma unroll 1
             for (int c = 0; c < BT / 32; ++c) {
                 if (m0 + 32 * c >= M) break;  // the rest of the tile lies past the last token (uniform)
@@ -388,8 +445,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
 
 template <class C>
 cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                       const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
-                       cudaStream_t s) {
+                       const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, int splits,
+                       int *tile_cnt, bool pdl, cudaStream_t s) {
     CUtensorMap ta, tw, to;
     if (!make_tmap_u8_2d(&ta, codes, (uint64_t)K, (uint64_t)M, BK, C::BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -397,7 +454,8 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
         return cudaErrorInvalidValue;
     // The bulk-store epilogue needs a 16-byte row pitch and base, and a box that fits.
     memset(&to, 0, sizeof(to));
-    const bool store_ok = N % 4 == 0 && M >= OUT_TOKENS && N >= BW && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+    const bool store_ok = splits == 1 && N % 4 == 0 && M >= OUT_TOKENS && N >= BW &&
+                          (reinterpret_cast<uintptr_t>(out) & 15) == 0;
     const int tma_out = store_ok && make_tmap_f32_2d(&to, out, (uint64_t)N, (uint64_t)M, BW, OUT_TOKENS) ? 1 : 0;
     auto kern = gemm_tc_kernel<C>;
     static bool done[kMaxDevices] = {};
@@ -409,8 +467,8 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) done[dev] = true;
     }
-    const long tiles = (long)((N + BW - 1) / BW) * ((M + C::BT - 1) / C::BT);
-    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+    const long units = (long)((N + BW - 1) / BW) * ((M + C::BT - 1) / C::BT) * splits;
+    const int grid = (int)(units < sm_count() ? units : sm_count());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(C::THREADS);
@@ -422,22 +480,26 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, packed, scale_x, alpha, mode, M, N, K, out, acc_out,
-                              device_status_ptr());
+                              splits, tile_cnt, device_status_ptr());
 }
 
 }  // namespace
 
-// Modelled time of one token-tile size, in units of one 128-k stage of one tile:
-// rounds of tiles per SM x (stages per tile x relative stage cost + a drain stall
-// per tile when the accumulator is single-buffered).  The stage costs and the
-// stall are B200 measurements: a stage takes about as long at 192..256 tokens,
-// and the single-buffered 256-token tile stalls about 10 stages per tile.
-double gemm_tile_cost(int bt, int M, int N, int K, int sms) {
+// Modelled time of a (token tile, k-split) choice, in units of one 128-k stage of one
+// tile: rounds of work units per SM x (stages per unit x relative stage cost + a
+// drain stall per unit when the accumulator is single-buffered + the split-K
+// epilogue).  All constants are B200 measurements: a stage takes about as long at
+// 192..256 tokens; the single-buffered 256-token tile stalls about 10 stages per
+// tile; a split tile costs about 20 + BT/4 stages more (the atomic additions, and
+// the last split dequantising the whole tile), so splitting only pays for few
+// output tiles and long K.
+double gemm_tile_cost(int bt, int splits, int M, int N, int K, int sms) {
     const double w = bt >= 192 ? 1.0 : (bt >= 128 ? 0.93 : 0.81);
     const double drain = bt == 256 ? 10.0 : 0.0;
-    const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
-    const long rounds = (tiles + sms - 1) / sms;
-    return (double)rounds * ((double)(K / BK) * w + drain);
+    const double split_cost = splits == 1 ? 0.0 : 20.0 + bt / 4.0;
+    const long units = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt) * splits;
+    const long rounds = (units + sms - 1) / sms;
+    return (double)rounds * ((double)(K / BK / splits) * w + drain + split_cost);
 }
 
 namespace {
@@ -450,30 +512,42 @@ bool gemm_force_tile(int bt) {
     return true;
 }
 
-int gemm_pick_tile(int M, int N, int K, int sms) {
-    if (g_forced_tile) return g_forced_tile;
-    static const int cand[] = {224, 192, 128, 64};
-    int best = 256;
-    double best_cost = gemm_tile_cost(256, M, N, K, sms);
-    for (int bt : cand) {
-        const double c = gemm_tile_cost(bt, M, N, K, sms);
-        if (c < best_cost * 0.999) {
-            best = bt;
-            best_cost = c;
+GemmPlan gemm_plan(int M, int N, int K, int sms, int max_split_tiles) {
+    static const int tiles_c[] = {256, 224, 192, 128, 64};
+    static const int splits_c[] = {1, 2, 4, 8};
+    GemmPlan best{256, 1};
+    double best_cost = 1e300;
+    const int KB = K / BK;
+    for (int bt : tiles_c) {
+        if (g_forced_tile && bt != g_forced_tile) continue;
+        const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
+        for (int sp : splits_c) {
+            if (sp > 1 && (tiles > max_split_tiles || KB % sp != 0 || KB / sp < 4)) continue;
+            const double c = gemm_tile_cost(bt, sp, M, N, K, sms);
+            if (c < best_cost * 0.999) {
+                best = GemmPlan{bt, sp};
+                best_cost = c;
+            }
         }
     }
     return best;
 }
 
+int gemm_pick_tile(int M, int N, int K, int sms) { return gemm_plan(M, N, K, sms, 0).token_tile; }
+
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                            const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
-                           cudaStream_t s) {
-    switch (gemm_pick_tile(M, N, K, sm_count())) {
-    case 256: return launch_cfg<Cfg256>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    case 224: return launch_cfg<Cfg224>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    case 192: return launch_cfg<Cfg192>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    case 128: return launch_cfg<Cfg128>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
-    default: return launch_cfg<Cfg64>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, pdl, s);
+                           cudaStream_t s, GemmPlan plan, int *tile_cnt) {
+    if (plan.token_tile == 0) plan = gemm_plan(M, N, K, sm_count(), 0);
+    const int sp = plan.splits;
+    if (sp < 1 || (sp > 1 && (!tile_cnt || (K / BK) % sp != 0))) return cudaErrorInvalidValue;
+    switch (plan.token_tile) {
+    case 256: return launch_cfg<Cfg256>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    case 224: return launch_cfg<Cfg224>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    case 192: return launch_cfg<Cfg192>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    case 128: return launch_cfg<Cfg128>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    case 64: return launch_cfg<Cfg64>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    default: return cudaErrorInvalidValue;
     }
 }
 

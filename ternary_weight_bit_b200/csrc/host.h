@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/bitnet.h"
+
 namespace bitnet {
 
 // Forwards and GEMMs with at most this many tokens run the decode kernel (gemv.cu);
@@ -28,8 +30,17 @@ int *device_status_ptr();
 // Number of SMs of the current device (cached).
 int sm_count();
 
+// Optional work for act_quant on behalf of a following split-K GEMM: zero `row_words`
+// 32-bit words per token row of `rows` (the GEMM output) and `cnt_n` tile counters.
+struct ZeroFill {
+    uint32_t *rows = nullptr;
+    int row_words = 0;
+    int *cnt = nullptr;
+    int cnt_n = 0;
+};
 cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
-                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s);
+                             int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s,
+                             ZeroFill zf = ZeroFill());
 
 size_t pack_workspace_bytes();
 cudaError_t launch_pack(const float *W, int64_t N, int64_t K, float eps, uint8_t *packed, float *alpha,
@@ -42,16 +53,33 @@ cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, con
                         bool pdl, cudaStream_t s);
 
 // Prefill path: tcgen05 int8 tensor-core GEMM with TMEM accumulators.
+// A plan is a token-tile size (256/224/192/128/64) and a k-split count (1, 2, 4, 8).
+// With splits > 1, `out` must be zero on entry (the kernel adds int32 partial sums
+// into it before dequantising in place) and tile_cnt must point at
+// kSplitCounters zeroed ints (the kernel leaves them zero again).
+struct GemmPlan {
+    int token_tile;  // 0: choose automatically (no split)
+    int splits;
+};
+constexpr int kSplitCounters = 1024;
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                            const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
-                           bool pdl, cudaStream_t s);
+                           bool pdl, cudaStream_t s, GemmPlan plan = GemmPlan{0, 1}, int *tile_cnt = nullptr);
 
-// Token-tile size launch_gemm_tc uses for this shape on `sms` SMs (256/224/192/128/64,
-// or the forced value), and the modelled cost the automatic choice compares.
+// The plan launch_gemm_tc uses for this shape on `sms` SMs; splits > 1 only when the
+// output has at most max_split_tiles tiles (0: never split).  Honors a forced tile.
+GemmPlan gemm_plan(int M, int N, int K, int sms, int max_split_tiles);
+// Token-tile size of the unsplit plan, and the modelled cost the choice compares.
 int gemm_pick_tile(int M, int N, int K, int sms);
-double gemm_tile_cost(int bt, int M, int N, int K, int sms);
+double gemm_tile_cost(int bt, int splits, int M, int N, int K, int sms);
 // Force the token tile (0 = automatic); false for an unsupported value.
 bool gemm_force_tile(int bt);
+
+// The forward's kernels (act_quant, then GEMV or GEMM), arguments validated;
+// tile_cnt points at kSplitCounters ints of workspace for a split-K GEMM.
+cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
+                            int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
+                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s);
 
 // Launch the timeout self-test kernel.
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);

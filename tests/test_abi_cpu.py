@@ -40,6 +40,9 @@ def test_gemm_token_tile_host_logic(L):
     assert L.bitnet_gemm_token_tile(-1, 256, 256) == -1
     assert L.bitnet_gemm_token_tile(64, 0, 256) == -1
     assert L.bitnet_gemm_token_tile(64, 256, 100) == -1
+    sp = ctypes.c_int(-5)
+    assert L.bitnet_forward_gemm_plan(8, 2560, 6912, ctypes.byref(sp)) == 0 and sp.value == 0
+    assert L.bitnet_forward_gemm_plan(64, 0, 256, ctypes.byref(sp)) == -1
     for bad in (1, 32, 96, 160, 255, 257, 512, -64):
         assert L.bitnet_gemm_force_token_tile(bad) == _native.ERR_INVALID_ARG
     try:
@@ -51,10 +54,11 @@ def test_gemm_token_tile_host_logic(L):
 
 
 def test_workspace_sizes(L):
+    cnt = 4096  # split-K tile counters
     assert L.bitnet_forward_workspace_bytes(0, 256) == 0
-    assert L.bitnet_forward_workspace_bytes(1, 256) == 256 + 256
-    assert L.bitnet_forward_workspace_bytes(3, 2560) == 7680 + 256
-    assert L.bitnet_forward_workspace_bytes(100, 128) == 12800 + 512
+    assert L.bitnet_forward_workspace_bytes(1, 256) == 256 + 256 + cnt
+    assert L.bitnet_forward_workspace_bytes(3, 2560) == 7680 + 256 + cnt
+    assert L.bitnet_forward_workspace_bytes(100, 128) == 12800 + 512 + cnt
     assert L.bitnet_pack_workspace_bytes(6912, 2560) >= 8 * 1184
 
 

@@ -207,7 +207,7 @@ def _forward_case(case, sample_rows=None):
     W = case.W.to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(W, eps=case.eps)
     out = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, case.N, eps=case.eps, fwht=case.fwht, mode=case.mode)
-    codes, _ = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=case.fwht, mode=case.mode)
+    codes, gscale = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=case.fwht, mode=case.mode)
     torch.cuda.synchronize()
     rows = np.arange(case.M) if sample_rows is None else sample_rows
     X32 = case.X.float().numpy()[rows]
@@ -220,8 +220,10 @@ def _forward_case(case, sample_rows=None):
     gcodes = host(codes)[rows]
     parity.check_codes(gcodes, r.codes, sh, case.name)
     gout = host(out)[rows]
-    # same codes -> same output (up to the per-token scale's last bits)
-    out_same = ref.dequant(ref.gemm_packed(gcodes, p_ref, case.N), r.scale_x, a_ref, mode)
+    gs = host(gscale)[rows]
+    parity.check_scale_bound(gs, r.scale_x, case.K, mode, case.name)
+    # same codes and scales -> identical output (exact accumulators, same IEEE steps)
+    out_same = ref.dequant(ref.gemm_packed(gcodes, p_ref, case.N), gs, a_ref, mode)
     parity.check_out_same_codes(gout, out_same, case.name)
     parity.check_out_end_to_end(gout, r.out, gcodes, r.codes, r.scale_x, a_ref, mode, case.name)
 
@@ -247,6 +249,44 @@ def test_forward_ragged(M, K, N, mode, fwht, xdt):
     case = synthetic.make_case("ragged", M, K, N, x_kind="student_t3", outliers=max(1, K // 100),
                                outlier_gain=50.0, x_dtype=xdt, fwht=fwht, mode=mode, seed=M + K)
     _forward_case(case)
+
+
+def _split_k_case(M, K, N, mode, fwht, seed):
+    case = synthetic.make_case("splitk", M, K, N, x_kind="student_t3", outliers=max(1, K // 100), outlier_gain=50.0,
+                               x_dtype="f32", fwht=fwht, mode=mode, seed=seed)
+    _forward_case(case)  # against the oracle
+    # bit-identical to the unsplit GEMM on the same codes
+    Xd = case.X.to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(case.W.to(DEV), eps=case.eps)
+    out = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, N, eps=case.eps, fwht=fwht, mode=mode)
+    codes, scale = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=fwht, mode=mode)
+    out_unsplit = tb.bitnet_ternary_gemm(codes, scale, mode, packed, alpha, N)
+    assert torch.equal(out, out_unsplit)
+    assert tb.bitnet_get_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,N,mode,fwht,splits", [
+    (40, 16384, 1000, "int8", False, 8),  # ragged tokens and weight rows
+    (33, 8192, 4096, "int4", True, 4),
+    (64, 16384, 2048, "int8", False, 8),
+    (128, 8192, 2048, "int4", True, 4),
+])
+def test_forward_split_k(M, K, N, mode, fwht, splits):
+    # few output tiles for the SMs: the forward splits K (int32 atomics into out)
+    assert tb.bitnet_forward_gemm_plan(M, N, K)[1] == splits
+    _split_k_case(M, K, N, mode, fwht, seed=M * 7 + K)
+
+
+@pytest.mark.parametrize("tile", [256, 224, 192, 128, 64])
+def test_forward_split_k_forced_tiles(tile):
+    try:
+        tb.bitnet_gemm_force_token_tile(tile)
+        M, K, N = 40, 16384, 1024
+        t, sp = tb.bitnet_forward_gemm_plan(M, N, K)
+        assert t == tile and sp > 1
+        _split_k_case(M, K, N, ("int8", "int4")[tile % 3 == 0], tile % 2 == 0, seed=tile)
+    finally:
+        tb.bitnet_gemm_force_token_tile(0)
 
 
 def _sample(M, n=32, seed=0):
