@@ -21,6 +21,8 @@
  *          tl2_lookup_simulation listing.
  *   [edge] "bitnet_cpp_edge.py": pack-once / forward-many (prepare_weights) and the
  *          claim that per-token integer kernels are lossless.
+ *   [v2] BitNetV2FFN.forward also defines the SwiGLU input of the down projection
+ *          (oracle_swiglu).
  *
  * Readings where the pages are silent or disagree (each one is listed in the
  * design notes with its reason):
@@ -32,6 +34,7 @@
  *   - The per-token scale returned is gamma (or beta) without eps (Eq. 5/6).
  *   - alpha = mean|W| is summed in double in index order, rounded once to float.
  *   - The dequant epilogue is out = (float)acc * ((alpha * scale_x) / Q).
+ *   - silu(g) = g / (1 + e^-g) in fp32 (the page calls F.silu = g * sigmoid(g)).
  */
 #include <math.h>
 #include <stdint.h>
@@ -163,6 +166,36 @@ int oracle_act_quant(const float *y, int64_t M, int64_t K, int mode, float eps,
  * it to tell a rounding near-tie, where two correct fp32 evaluation orders may
  * land on different codes, from a real disagreement.
  * ------------------------------------------------------------------------- */
+/* Steps 1-3 in double on one token row (overwritten), pre-rounding values into v. */
+static void shadow_row(double *row, int64_t K, const float *g, double eps, int fwht, int mode, double *v)
+{
+    const double c = 1.0 / sqrt(2.0);
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) ss += row[k] * row[k];
+    double r = 1.0 / sqrt(ss / (double)K + eps);
+    for (int64_t k = 0; k < K; ++k) row[k] = row[k] * r * (g ? (double)g[k] : 1.0);
+    if (fwht) {
+        for (int64_t h = 1; h < K; h *= 2)
+            for (int64_t j0 = 0; j0 < K; j0 += 2 * h)
+                for (int64_t j = j0; j < j0 + h; ++j) {
+                    double a = row[j], b = row[j + h];
+                    row[j] = (a + b) * c;
+                    row[j + h] = (a - b) * c;
+                }
+    }
+    double s;
+    if (mode == ORACLE_ACT_INT8) {
+        double gamma = 0.0;
+        for (int64_t k = 0; k < K; ++k) gamma = fabs(row[k]) > gamma ? fabs(row[k]) : gamma;
+        s = 127.0 / (gamma + eps);
+    } else {
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k) sum += fabs(row[k]);
+        s = sqrt(7.0) / (sum / (double)K + eps);
+    }
+    for (int64_t k = 0; k < K; ++k) v[k] = row[k] * s;
+}
+
 int oracle_shadow_prerounding(const float *x, int64_t M, int64_t K, const float *g,
                               double eps, int fwht, int mode, double *v)
 {
@@ -170,33 +203,46 @@ int oracle_shadow_prerounding(const float *x, int64_t M, int64_t K, const float 
     if (fwht && !is_pow2(K)) return ORACLE_NOT_POW2;
     double *row = (double *)malloc((size_t)K * sizeof(double));
     if (!row) return ORACLE_BAD_ARG;
-    const double c = 1.0 / sqrt(2.0);
     for (int64_t m = 0; m < M; ++m) {
-        const float *xr = x + m * K;
-        double ss = 0.0;
-        for (int64_t k = 0; k < K; ++k) ss += (double)xr[k] * (double)xr[k];
-        double r = 1.0 / sqrt(ss / (double)K + eps);
-        for (int64_t k = 0; k < K; ++k) row[k] = (double)xr[k] * r * (g ? (double)g[k] : 1.0);
-        if (fwht) {
-            for (int64_t h = 1; h < K; h *= 2)
-                for (int64_t j0 = 0; j0 < K; j0 += 2 * h)
-                    for (int64_t j = j0; j < j0 + h; ++j) {
-                        double a = row[j], b = row[j + h];
-                        row[j] = (a + b) * c;
-                        row[j + h] = (a - b) * c;
-                    }
+        for (int64_t k = 0; k < K; ++k) row[k] = (double)x[m * K + k];
+        shadow_row(row, K, g, eps, fwht, mode, v + m * K);
+    }
+    free(row);
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * SwiGLU input of the FFN down projection.  [v2] BitNetV2FFN.forward:
+ *   gate = F.silu(gate_proj(x)); up = up_proj(x); inter = gate * up
+ * with silu(g) = g * sigmoid(g) = g / (1 + e^-g), here one fp32 rounding per
+ * operation:  inter = (g / (1.0f + expf(-g))) * u.
+ * ------------------------------------------------------------------------- */
+int oracle_swiglu(const float *gate, const float *up, int64_t count, float *out)
+{
+    if (count < 0) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < count; ++i) {
+        float gv = gate[i];
+        float den = 1.0f + expf(-gv);
+        float silu = gv / den;
+        out[i] = silu * up[i];
+    }
+    return ORACLE_OK;
+}
+
+/* fp64 shadow of the SwiGLU product followed by steps 1-3 (see oracle_shadow_prerounding). */
+int oracle_shadow_swiglu(const float *gate, const float *up, int64_t M, int64_t K, const float *g,
+                         double eps, int fwht, int mode, double *v)
+{
+    if (K <= 0 || M < 0) return ORACLE_BAD_ARG;
+    if (fwht && !is_pow2(K)) return ORACLE_NOT_POW2;
+    double *row = (double *)malloc((size_t)K * sizeof(double));
+    if (!row) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) {
+            double gv = (double)gate[m * K + k];
+            row[k] = gv / (1.0 + exp(-gv)) * (double)up[m * K + k];
         }
-        double s;
-        if (mode == ORACLE_ACT_INT8) {
-            double gamma = 0.0;
-            for (int64_t k = 0; k < K; ++k) gamma = fabs(row[k]) > gamma ? fabs(row[k]) : gamma;
-            s = 127.0 / (gamma + eps);
-        } else {
-            double sum = 0.0;
-            for (int64_t k = 0; k < K; ++k) sum += fabs(row[k]);
-            s = sqrt(7.0) / (sum / (double)K + eps);
-        }
-        for (int64_t k = 0; k < K; ++k) v[m * K + k] = row[k] * s;
+        shadow_row(row, K, g, eps, fwht, mode, v + m * K);
     }
     free(row);
     return ORACLE_OK;

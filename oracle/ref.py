@@ -51,9 +51,11 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_gemm_int.argtypes = [P, P, I64, I64, I64, P]
     L.oracle_gemm_packed.argtypes = [P, P, I64, I64, I64, P]
     L.oracle_dequant.argtypes = [P, P, F, I, I64, I64, P]
+    L.oracle_swiglu.argtypes = [P, P, I64, P]
+    L.oracle_shadow_swiglu.argtypes = [P, P, I64, I64, P, D, I, I, P]
     for name in ("oracle_rmsnorm", "oracle_fwht", "oracle_act_quant", "oracle_shadow_prerounding",
                  "oracle_ternarize", "oracle_pack", "oracle_unpack", "oracle_gemm_int",
-                 "oracle_gemm_packed", "oracle_dequant"):
+                 "oracle_gemm_packed", "oracle_dequant", "oracle_swiglu", "oracle_shadow_swiglu"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -125,6 +127,31 @@ def shadow(x, g=None, eps: float = 1e-5, fwht_on: bool = False, mode: int = ACT_
     gp = None if g is None else _f32(g)
     _check("shadow", L.oracle_shadow_prerounding(_p(x), M, K, None if gp is None else _p(gp),
                                                  float(np.float32(eps)), int(fwht_on), mode, _p(v)))
+    return v
+
+
+def swiglu(gate, up, L=None) -> np.ndarray:
+    """SwiGLU input of the FFN down projection: silu(gate) * up, fp32 (same shape)."""
+    L = L or lib()
+    g = _f32(gate)
+    u = _f32(up)
+    assert g.shape == u.shape
+    out = np.empty_like(g)
+    _check("swiglu", L.oracle_swiglu(_p(g), _p(u), g.size, _p(out)))
+    return out
+
+
+def shadow_swiglu(gate, up, g=None, eps: float = 1e-5, fwht_on: bool = False, mode: int = ACT_INT8,
+                  L=None) -> np.ndarray:
+    """fp64 pre-rounding value of every activation code of the SwiGLU input."""
+    L = L or lib()
+    ga = _f32(gate)
+    u = _f32(up)
+    M, K = ga.shape
+    v = np.empty((M, K), dtype=np.float64)
+    gp = None if g is None else _f32(g)
+    _check("shadow_swiglu", L.oracle_shadow_swiglu(_p(ga), _p(u), M, K, None if gp is None else _p(gp),
+                                                   float(np.float32(eps)), int(fwht_on), mode, _p(v)))
     return v
 
 

@@ -33,6 +33,9 @@ MUTANTS = {
                               "s += (int32_t)q[m * K + k] * (int32_t)(code);"),
     "alpha_sum_not_mean": ("return (float)(sum / (double)count);", "return (float)(sum);"),
     "dequant_times_q": ("float f = (alpha * scale_x[m]) / Q;", "float f = (alpha * scale_x[m]) * Q;"),
+    "swiglu_sigmoid_only": ("float silu = gv / den;", "float silu = 1.0f / den;"),
+    "swiglu_wrong_exp_sign": ("float den = 1.0f + expf(-gv);", "float den = 1.0f + expf(gv);"),
+    "swiglu_drops_up": ("out[i] = silu * up[i];", "out[i] = silu;"),
 }
 
 

@@ -276,3 +276,59 @@ def test_hand_cases(mode_name):
         np.testing.assert_allclose(s[0], exp["scale"], rtol=2e-6)
         assert acc[0].tolist() == exp["acc"]
         np.testing.assert_allclose(out[0], exp["out"], rtol=2e-6, atol=1e-9)
+
+
+# ----------------------------------------------------------------------------- SwiGLU input
+# (bitnet_v2_engine.py page, BitNetV2FFN.forward: silu(gate_proj(x)) * up_proj(x))
+def _ulp_rel(a, b):
+    return abs(float(a) - float(b)) / max(abs(float(b)), 1e-30)
+
+
+def test_swiglu_closed_form_values():
+    gate = np.array([[0.0, 1.0, -1.0, 2.0, 50.0, -100.0, 20.0]], np.float32)
+    up = np.array([[3.0, 1.0, 2.0, 0.5, 2.0, 5.0, 1.0]], np.float32)
+    got = ref.swiglu(gate, up)[0]
+    assert got[0] == 0.0                                       # silu(0) = 0
+    assert _ulp_rel(got[1], 1.0 / (1.0 + math.exp(-1.0))) < 3e-7  # sigmoid(1)
+    assert _ulp_rel(got[2], -2.0 / (1.0 + math.e)) < 3e-7      # 2 * silu(-1) = -2 / (1 + e)
+    assert _ulp_rel(got[3], 1.0 / (1.0 + math.exp(-2.0))) < 3e-7  # 0.5 * silu(2) = sigmoid(2)
+    assert got[4] == 100.0                                     # e^-50 vanishes against 1
+    assert got[5] == 0.0 and math.copysign(1.0, got[5]) < 0   # -100 / inf = -0
+    assert got[6] == 20.0                                      # sigmoid(20) rounds to 1 in fp32
+
+
+def test_swiglu_odd_part_is_the_identity():
+    # silu(x) - silu(-x) = x (sigmoid(x) + sigmoid(-x) = 1)
+    x = np.random.default_rng(5).uniform(-12, 12, size=4000).astype(np.float32)
+    ones = np.ones_like(x)
+    d = ref.swiglu(x[None], ones[None])[0].astype(np.float64) - ref.swiglu(-x[None], ones[None])[0]
+    np.testing.assert_allclose(d, x.astype(np.float64), rtol=2e-6, atol=1e-6)
+
+
+def test_swiglu_minimum_is_minus_lambert_w_of_inverse_e():
+    # min_x x*sigmoid(x) = -W(1/e) at x = -1 - W(1/e) (W: Lambert W, principal branch)
+    w = 0.27846454276107380  # W(e^-1), the solution of w e^w = e^-1
+    x = np.arange(-3.0, 0.0, 1e-3, dtype=np.float64).astype(np.float32)
+    f = ref.swiglu(x[None], np.ones_like(x)[None])[0]
+    assert abs(float(f.min()) + w) < 2e-6
+    assert abs(float(x[np.argmin(f)]) + 1.0 + w) < 2e-3
+
+
+def test_swiglu_scales_exactly_with_up():
+    g = np.random.default_rng(6).normal(0, 3, size=(4, 64)).astype(np.float32)
+    one = ref.swiglu(g, np.ones_like(g))
+    for p2 in (0.25, 4.0, -8.0):
+        np.testing.assert_array_equal(ref.swiglu(g, np.full_like(g, p2)), one * np.float32(p2))
+
+
+def test_shadow_swiglu_agrees_with_fp32_codes_away_from_ties():
+    rng = np.random.default_rng(7)
+    gate = rng.normal(0, 2, size=(6, 512)).astype(np.float32)
+    up = rng.normal(0, 1, size=(6, 512)).astype(np.float32)
+    for mode in (ref.ACT_INT8, ref.ACT_INT4):
+        q, _ = ref.act_quant(ref.swiglu(gate, up), eps=1e-5, fwht_on=True, mode=mode)
+        v = ref.shadow_swiglu(gate, up, eps=1e-5, fwht_on=True, mode=mode)
+        lo, hi = (-128, 127) if mode == ref.ACT_INT8 else (-8, 7)
+        want = np.clip(np.rint(v), lo, hi)
+        far = np.abs(v - np.floor(v) - 0.5) > 1e-3
+        np.testing.assert_array_equal(q[far], want[far])
