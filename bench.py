@@ -55,6 +55,8 @@ def workload_cases(name: str):
         return cases
     if name == "wdown":
         return [("wdown", 2048, 2048, 8192, "int4", True, "student_t3", "f32", 82)]
+    if name == "wdown_swiglu":
+        return [("wdown_swiglu", 2048, 2048, 8192, "int4", True, "swiglu", "f32", 0)]
     m = re.fullmatch(r"msweep_M(\d+)", name)
     if m:
         M = int(m.group(1))
@@ -68,6 +70,8 @@ WORKLOAD_TEXT = {
               "[6912x2560] and [2560x6912] (N(0,0.02) absmean-ternarised, 2-bit packed); 6 forwards per step",
     "prefill": "prefill int8, 7B-like projections: X bf16 [4096,4096]; W Wq/Wk/Wv/Wo [4096x4096] (FWHT on Wo only) "
                "and Wup/Wgate [11008x4096]; 6 forwards per step",
+    "wdown_swiglu": "FFN down projection fused with its SwiGLU input: gate N(0,2^2) and up N(0,1) [2048,8192] "
+                    "-> silu(gate)*up formed in the activation kernel -> int4 absmean + FWHT; W [2048x8192]",
     "wdown": "Wdown-style H-BitLinear, int4 absmean + FWHT: X Student-t(3) [2048,8192] with 1% channels x50; "
              "W [2048x8192]",
 }
@@ -234,6 +238,8 @@ def time_oracle(cases, budget_s: float, steps: int | None = None):
             ncols = max(1, min(c.N, int(math.ceil(c.N * frac))))
             X = c.X.float().numpy()
             t0 = time.perf_counter()
+            if c.up is not None:
+                X = ref.swiglu(X, c.up.float().numpy())
             q, s = ref.act_quant(X, None, c.eps, c.fwht, mode)
             t1 = time.perf_counter()
             acc = ref.gemm_packed(q, packed[:ncols], ncols)
@@ -281,23 +287,34 @@ def run_ours(args):
         del W
         base.append((packed, alpha))
     packed_bytes = sum(p.numel() for p, _ in base)
-    step_bytes = packed_bytes + sum(c.X.numel() * c.X.element_size() for c in host)
+    def in_bytes(c):
+        return c.X.numel() * c.X.element_size() * (2 if c.up is not None else 1)
+
+    step_bytes = packed_bytes + sum(in_bytes(c) for c in host)
     R = max(1, min(64, math.ceil(4 * l2 / step_bytes))) if step_bytes < 4 * l2 else 1
-    rot = []  # R copies of (X, packed, alpha, out, ws) per case
+    rot = []  # R copies of (X, packed, alpha, out, ws, up) per case
     for r in range(R):
         items = []
         for c, (p, a) in zip(host, base):
             X = c.X.to(dev)
+            U = None if c.up is None else c.up.to(dev)
             ws = torch.empty((max(tb.bitnet_forward_workspace_bytes(c.M, c.K), 256),), dtype=torch.uint8,
                              device=dev)
             out = torch.empty((c.M, c.N), dtype=torch.float32, device=dev)
-            items.append((X, p.clone() if r else p, a, out, ws))
+            items.append((X, p.clone() if r else p, a, out, ws, U))
         rot.append(items)
     torch.cuda.synchronize()
 
-    def step(r):
-        for c, (X, p, a, out, ws) in zip(host, rot[r]):
+    def forward(c, X, p, a, out, ws, U):
+        if U is None:
             tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+        else:
+            tb.bitnet_hbitlinear_forward_swiglu(X, U, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out,
+                                                ws=ws)
+
+    def step(r):
+        for c, item in zip(host, rot[r]):
+            forward(c, *item)
 
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
@@ -354,13 +371,16 @@ def run_ours(args):
 
     # ------------------------------------------------------------------ dominant kernel alone
     codes_scales = []
-    for c, (X, p, a, out, ws) in zip(host, rot[0]):
-        codes, scale = tb.bitnet_act_quant(X, eps=c.eps, fwht=c.fwht, mode=c.mode)
+    for c, (X, p, a, out, ws, U) in zip(host, rot[0]):
+        if U is None:
+            codes, scale = tb.bitnet_act_quant(X, eps=c.eps, fwht=c.fwht, mode=c.mode)
+        else:
+            codes, scale = tb.bitnet_act_quant_swiglu(X, U, eps=c.eps, fwht=c.fwht, mode=c.mode)
         codes_scales.append((codes, scale))
     torch.cuda.synchronize(dev)
 
     def gemm_pass(r):
-        for c, (codes, scale), (X, p, a, out, ws) in zip(host, codes_scales, rot[r]):
+        for c, (codes, scale), (X, p, a, out, ws, U) in zip(host, codes_scales, rot[r]):
             tb.bitnet_ternary_gemm(codes, scale, c.mode, p, a, c.N, out=out)
 
     gg = torch.cuda.CUDAGraph()
@@ -414,13 +434,16 @@ def run_ours(args):
 
     # ------------------------------------------------------------------ end to end through the public API
     pinned_x = [c.X.pin_memory() for c in host]
+    pinned_u = [None if c.up is None else c.up.pin_memory() for c in host]
     pinned_o = [torch.empty((c.M, c.N), dtype=torch.float32).pin_memory() for c in host]
     e2e_steps = max(3, min(args.steps, 200))
     with torch.cuda.stream(stream):
         for _ in range(2):
-            for c, hx, ho, (X, p, a, out, ws) in zip(host, pinned_x, pinned_o, rot[0]):
+            for c, hx, hu, ho, (X, p, a, out, ws, U) in zip(host, pinned_x, pinned_u, pinned_o, rot[0]):
                 X.copy_(hx, non_blocking=True)
-                tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+                if U is not None:
+                    U.copy_(hu, non_blocking=True)
+                forward(c, X, p, a, out, ws, U)
                 ho.copy_(out, non_blocking=True)
     stream.synchronize()
     x0 = torch.cuda.Event(enable_timing=True)
@@ -428,15 +451,17 @@ def run_ours(args):
     x0.record(stream)
     with torch.cuda.stream(stream):
         for i in range(e2e_steps):
-            for c, hx, ho, (X, p, a, out, ws) in zip(host, pinned_x, pinned_o, rot[i % R]):
+            for c, hx, hu, ho, (X, p, a, out, ws, U) in zip(host, pinned_x, pinned_u, pinned_o, rot[i % R]):
                 X.copy_(hx, non_blocking=True)
-                tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+                if U is not None:
+                    U.copy_(hu, non_blocking=True)
+                forward(c, X, p, a, out, ws, U)
                 ho.copy_(out, non_blocking=True)
     x1.record(stream)
     x1.synchronize()
     e2e_ms = x0.elapsed_time(x1)
     e2e_max, e2e_tokens = aggregate(e2e_ms, e2e_steps * sum(c.M for c in host), world, dev)
-    h2d = sum(c.X.numel() * c.X.element_size() for c in host)
+    h2d = sum(in_bytes(c) for c in host)
     d2h = sum(4 * c.M * c.N for c in host)
 
     result = None
@@ -456,7 +481,7 @@ def run_ours(args):
             "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
             "e2e": {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "note": "eager calls of bitnet_hbitlinear_forward with pinned host X in and out per step"},
+                    "note": "eager calls of the public forward with pinned host inputs in and output out per step"},
             "gpu_launches": args.steps * 2 * len(host),
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
             "device_status": status,

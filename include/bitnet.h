@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 2
+#define BITNET_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -167,6 +167,29 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype
                                           bitnet_act_mode_t mode, const uint8_t *packed,
                                           const float *alpha, int64_t N, float *out,
                                           void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * SwiGLU-fused variants for the down projection of a BitNet v2 FFN.
+ * Definition: bitnet_v2_engine.py page, BitNetV2FFN.forward:
+ *   inter = F.silu(gate_proj(x)) * up_proj(x);  out = down_proj(inter)
+ * with down_proj an H-BitLinear.  Here the activation step reads gate and up and
+ * forms, elementwise in fp32 with one IEEE rounding per operation,
+ *   inter[m][k] = (gate / (1 + exp(-gate))) * up        (exp: CUDA expf)
+ * in registers; inter is then normalised, rotated and quantised exactly as X is
+ * in bitnet_act_quant, and never written to memory.
+ *   gate, up  [M][K] in dtype xdt, device, read only (16-byte aligned).
+ *   Other arguments, results and errors as for bitnet_act_quant and
+ *   bitnet_hbitlinear_forward (the workspace is the same size).
+ * ------------------------------------------------------------------------ */
+BITNET_API bitnet_status_t bitnet_act_quant_swiglu(const void *gate, const void *up, bitnet_dtype_t xdt, int64_t M,
+                                                   int64_t K, const float *gain, float eps, int fwht,
+                                                   bitnet_act_mode_t mode, int8_t *codes, float *scale_x,
+                                                   void *stream);
+BITNET_API bitnet_status_t bitnet_hbitlinear_forward_swiglu(const void *gate, const void *up, bitnet_dtype_t xdt,
+                                                            int64_t M, int64_t K, const float *gain, float eps,
+                                                            int fwht, bitnet_act_mode_t mode, const uint8_t *packed,
+                                                            const float *alpha, int64_t N, float *out, void *ws,
+                                                            size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * bitnet_hbitlinear_forward_noalloc -- the same forward as bitnet_hbitlinear_forward,

@@ -26,6 +26,7 @@ __all__ = [
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
     "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_forward_gemm_plan",
+    "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu",
 ]
 
 _MODES = {"int8": _native.ACT_INT8_ABSMAX, "int4": _native.ACT_INT4_ABSMEAN}
@@ -135,6 +136,53 @@ def bitnet_act_quant(X: torch.Tensor, gain=None, eps: float = 1e-5, fwht: bool =
                   L.bitnet_act_quant(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)), mode_id(mode),
                                      _ptr(codes), _ptr(scale_x), _stream(stream)))
     return codes, scale_x
+
+
+def _need_pair(gate: torch.Tensor, up: torch.Tensor) -> None:
+    _need(gate, "gate")
+    _need(up, "up", gate.dtype, tuple(gate.shape))
+
+
+def bitnet_act_quant_swiglu(gate: torch.Tensor, up: torch.Tensor, gain=None, eps: float = 1e-5, fwht: bool = True,
+                            mode="int4", codes=None, scale_x=None, stream=None):
+    """bitnet_act_quant on the SwiGLU product silu(gate) * up (formed in registers, never stored).
+    Returns (codes int8 [M,K], scale fp32 [M])."""
+    L = _native.load()
+    _need_pair(gate, up)
+    M, K = gate.shape
+    codes = torch.empty((M, K), dtype=torch.int8, device=gate.device) if codes is None else codes
+    scale_x = torch.empty((M,), dtype=torch.float32, device=gate.device) if scale_x is None else scale_x
+    _need(codes, "codes", torch.int8, (M, K))
+    _need(scale_x, "scale_x", torch.float32, (M,))
+    if gain is not None:
+        _need(gain, "gain", torch.float32, (K,))
+    _native.check("bitnet_act_quant_swiglu",
+                  L.bitnet_act_quant_swiglu(_ptr(gate), _ptr(up), _xdt(gate), M, K, _ptr(gain), eps, int(bool(fwht)),
+                                            mode_id(mode), _ptr(codes), _ptr(scale_x), _stream(stream)))
+    return codes, scale_x
+
+
+def bitnet_hbitlinear_forward_swiglu(gate: torch.Tensor, up: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor,
+                                     N: int, gain=None, eps: float = 1e-5, fwht: bool = True, mode="int4", out=None,
+                                     ws=None, stream=None):
+    """The H-BitLinear down projection of a BitNet v2 FFN on silu(gate) * up.  Returns out fp32 [M, N]."""
+    L = _native.load()
+    _need_pair(gate, up)
+    M, K = gate.shape
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(alpha, "alpha", torch.float32)
+    if gain is not None:
+        _need(gain, "gain", torch.float32, (K,))
+    out = torch.empty((M, N), dtype=torch.float32, device=gate.device) if out is None else out
+    _need(out, "out", torch.float32, (M, N))
+    nbytes = L.bitnet_forward_workspace_bytes(M, K)
+    ws = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=gate.device) if ws is None else ws
+    _need(ws, "ws", torch.uint8)
+    _native.check("bitnet_hbitlinear_forward_swiglu",
+                  L.bitnet_hbitlinear_forward_swiglu(_ptr(gate), _ptr(up), _xdt(gate), M, K, _ptr(gain), eps,
+                                                     int(bool(fwht)), mode_id(mode), _ptr(packed), _ptr(alpha), N,
+                                                     _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 def bitnet_ternary_gemm(codes: torch.Tensor, scale_x: torch.Tensor, mode, packed: torch.Tensor,

@@ -143,6 +143,42 @@ __device__ __forceinline__ void load4(const void *X, int64_t idx, float *v) {
     }
 }
 
+// ------------------------------------------------------------------ input sources
+// The kernels read their per-token input through a source: XSrc reads X itself;
+// SwigluSrc forms the SwiGLU product silu(gate) * up of a BitNet v2 FFN on the fly
+// (bitnet_v2_engine.py page, BitNetV2FFN.forward: F.silu(gate_proj(x)) * up_proj(x)),
+// so the intermediate activation never makes an fp32 round trip through HBM.
+template <bool BF16>
+struct XSrc {
+    const void *X;
+    __device__ __forceinline__ void get8(int64_t idx, float *v) const { load8<BF16>(X, idx, v); }
+    __device__ __forceinline__ void get4(int64_t idx, float *v) const { load4<BF16>(X, idx, v); }
+};
+
+// silu(g) * u with silu(g) = g / (1 + e^-g), each step one IEEE rounding.
+__device__ __forceinline__ float swiglu(float g, float u) {
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+template <bool BF16>
+struct SwigluSrc {
+    const void *gate, *up;
+    __device__ __forceinline__ void get8(int64_t idx, float *v) const {
+        float u[8];
+        load8<BF16>(gate, idx, v);
+        load8<BF16>(up, idx, u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = swiglu(v[i], u[i]);
+    }
+    __device__ __forceinline__ void get4(int64_t idx, float *v) const {
+        float u[4];
+        load4<BF16>(gate, idx, v);
+        load4<BF16>(up, idx, u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = swiglu(v[i], u[i]);
+    }
+};
+
 // ------------------------------------------------------------------ FWHT kernel
 template <int LOGK>
 struct FwhtShape {
@@ -190,9 +226,9 @@ __device__ __forceinline__ void zero_fill(const ZeroFill &z) {
         for (int i = threadIdx.x; i < z.cnt_n; i += blockDim.x) z.cnt[i] = 0;
 }
 
-template <int LOGK, bool BF16>
+template <int LOGK, class Src>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::T)
-act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain, float eps, int mode,
+act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mode,
                       int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
     using S = FwhtShape<LOGK>;
     constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
@@ -213,9 +249,9 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
     // Phase 0 layout: thread tid owns the E contiguous elements [tid*E, tid*E + E).
     if constexpr (E >= 8) {
 #pragma unroll
-        for (int c = 0; c < E / 8; ++c) load8<BF16>(X, row + tid * E + 8 * c, v + 8 * c);
+        for (int c = 0; c < E / 8; ++c) src.get8(row + tid * E + 8 * c, v + 8 * c);
     } else {
-        load4<BF16>(X, row + tid * E, v);
+        src.get4(row + tid * E, v);
     }
 
     float ss = 0.0f;
@@ -310,9 +346,9 @@ act_quant_fwht_kernel(const void *__restrict__ X, const float *__restrict__ gain
 
 // ------------------------------------------------------------------ plain kernel (no FWHT)
 // Thread tid owns the float4 groups j = it*T + tid, it in [0, NV); K % 4 == 0.
-template <int T, int NV, bool BF16>
+template <int T, int NV, class Src>
 __global__ void __launch_bounds__(T)
-act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gain, int K, float eps,
+act_quant_plain_kernel(Src src, const float *__restrict__ gain, int K, float eps,
                        int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
     __shared__ float red[32];
     pdl_launch_dependents();  // as in the FWHT kernel: the GEMM may launch, X is waited for
@@ -327,7 +363,7 @@ act_quant_plain_kernel(const void *__restrict__ X, const float *__restrict__ gai
     for (int it = 0; it < NV; ++it) {
         const int j = it * T + tid;
         if (j < K4) {
-            load4<BF16>(X, row + 4 * j, v[it]);
+            src.get4(row + 4 * j, v[it]);
         } else {
             v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.0f;
         }
@@ -392,12 +428,12 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int LOGK, bool BF16>
-cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
+template <int LOGK, class Src>
+cudaError_t launch_fwht(const Src &src, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
                         float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     using S = FwhtShape<LOGK>;
     const size_t smem = (size_t)(S::K + S::K / 32) * sizeof(float);
-    auto kern = act_quant_fwht_kernel<LOGK, BF16>;
+    auto kern = act_quant_fwht_kernel<LOGK, Src>;
     if (smem > 48 * 1024) {
         static bool done[kMaxDevices] = {};
         int dev = 0;
@@ -409,52 +445,60 @@ cudaError_t launch_fwht(const void *X, int64_t M, const float *gain, float eps, 
             if (dev < kMaxDevices) done[dev] = true;
         }
     }
-    return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, X, gain, eps, mode, codes, scale_x, zf);
+    return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, src, gain, eps, mode, codes, scale_x, zf);
 }
 
-template <int NV, bool BF16>
-cudaError_t launch_plain(const void *X, int64_t M, int K, const float *gain, float eps, int mode,
+template <int NV, class Src>
+cudaError_t launch_plain(const Src &src, int64_t M, int K, const float *gain, float eps, int mode,
                          int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     constexpr int T = 256;
-    return launch_pdl(act_quant_plain_kernel<T, NV, BF16>, dim3((unsigned)M), dim3(T), 0, s, X, gain, K, eps, mode,
+    return launch_pdl(act_quant_plain_kernel<T, NV, Src>, dim3((unsigned)M), dim3(T), 0, s, src, gain, K, eps, mode,
                       codes, scale_x, zf);
 }
 
-template <bool BF16>
-cudaError_t dispatch(const void *X, int64_t M, int K, const float *gain, float eps, int fwht, int mode,
+template <class Src>
+cudaError_t dispatch(const Src &src, int64_t M, int K, const float *gain, float eps, int fwht, int mode,
                      int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     if (fwht) {
         switch (__builtin_ctz((unsigned)K)) {
-            case 7: return launch_fwht<7, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 8: return launch_fwht<8, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 9: return launch_fwht<9, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 10: return launch_fwht<10, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 11: return launch_fwht<11, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 12: return launch_fwht<12, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 13: return launch_fwht<13, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 14: return launch_fwht<14, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
-            case 15: return launch_fwht<15, BF16>(X, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 7: return launch_fwht<7>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 8: return launch_fwht<8>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 9: return launch_fwht<9>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 10: return launch_fwht<10>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 11: return launch_fwht<11>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 12: return launch_fwht<12>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 13: return launch_fwht<13>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 14: return launch_fwht<14>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+            case 15: return launch_fwht<15>(src, M, gain, eps, mode, codes, scale_x, zf, s);
             default: return cudaErrorInvalidValue;
         }
     }
     const int nv = (int)ceil_div(K / 4, 256);
-    if (nv <= 1) return launch_plain<1, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 2) return launch_plain<2, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 4) return launch_plain<4, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 8) return launch_plain<8, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 16) return launch_plain<16, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 32) return launch_plain<32, BF16>(X, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 1) return launch_plain<1>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 2) return launch_plain<2>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 4) return launch_plain<4>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 8) return launch_plain<8>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 16) return launch_plain<16>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv <= 32) return launch_plain<32>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Host entry used by the ABI layer (arguments already validated).
+// Host entries used by the ABI layer (arguments already validated).
 cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
                              int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s, ZeroFill zf) {
     if (M == 0) return cudaSuccess;
-    return bf16 ? dispatch<true>(X, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s)
-                : dispatch<false>(X, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s);
+    return bf16 ? dispatch(XSrc<true>{X}, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s)
+                : dispatch(XSrc<false>{X}, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s);
+}
+
+cudaError_t launch_act_quant_swiglu(const void *gate, const void *up, bool bf16, int64_t M, int K, const float *gain,
+                                    float eps, int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s,
+                                    ZeroFill zf) {
+    if (M == 0) return cudaSuccess;
+    return bf16 ? dispatch(SwigluSrc<true>{gate, up}, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s)
+                : dispatch(SwigluSrc<false>{gate, up}, M, K, gain, eps, fwht, mode, codes, scale_x, zf, s);
 }
 
 }  // namespace bitnet

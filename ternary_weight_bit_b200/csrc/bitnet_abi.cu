@@ -158,7 +158,8 @@ cudaError_t run_gemm(const int8_t *codes, const float *scale_x, int mode, const 
 // splits K: act_quant then also zeroes `out` and the tile counters for it.
 cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
                             int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
-                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s) {
+                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
+                            const void *up) {
     GemmPlan plan{0, 1};
     ZeroFill zf;
     if (M > kGemvMaxM) {
@@ -170,7 +171,9 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
             zf.cnt_n = (int)(((N + 127) / 128) * ((M + plan.token_tile - 1) / plan.token_tile));
         }
     }
-    cudaError_t e = launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s, zf);
+    cudaError_t e = up ? launch_act_quant_swiglu(X, up, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes,
+                                                 scale_x, s, zf)
+                       : launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s, zf);
     if (e != cudaSuccess) return e;
     if (M <= kGemvMaxM)
         return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s);
@@ -247,10 +250,10 @@ size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K) {
            (size_t)kSplitCounters * sizeof(int);
 }
 
-bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
-                                          const float *gain, float eps, int fwht, bitnet_act_mode_t mode,
-                                          const uint8_t *packed, const float *alpha, int64_t N, float *out,
-                                          void *ws, size_t ws_bytes, void *stream) {
+namespace {
+bitnet_status_t forward_ws(const void *X, const void *up, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                           const float *gain, float eps, int fwht, bitnet_act_mode_t mode, const uint8_t *packed,
+                           const float *alpha, int64_t N, float *out, void *ws, size_t ws_bytes, void *stream) {
     if (N < 1 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
     bitnet_status_t st = validate_act(X, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
     if (st != BITNET_OK || M == 0) return st;
@@ -262,7 +265,37 @@ bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int
     float *scale_x = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)M * (size_t)K));
     int *tile_cnt = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(scale_x) + align256((size_t)M * sizeof(float)));
     return from_cuda(forward_kernels(X, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, codes, scale_x,
-                                     tile_cnt, static_cast<cudaStream_t>(stream)));
+                                     tile_cnt, static_cast<cudaStream_t>(stream), up));
+}
+}  // namespace
+
+bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                          const float *gain, float eps, int fwht, bitnet_act_mode_t mode,
+                                          const uint8_t *packed, const float *alpha, int64_t N, float *out,
+                                          void *ws, size_t ws_bytes, void *stream) {
+    return forward_ws(X, nullptr, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, ws, ws_bytes, stream);
+}
+
+bitnet_status_t bitnet_act_quant_swiglu(const void *gate, const void *up, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                        const float *gain, float eps, int fwht, bitnet_act_mode_t mode, int8_t *codes,
+                                        float *scale_x, void *stream) {
+    bitnet_status_t st = validate_act(gate, xdt, M, K, gain, fwht, mode, codes, scale_x, true);
+    if (st != BITNET_OK || M == 0) return st;
+    if (!up || !aligned16(up)) return BITNET_ERR_INVALID_ARG;
+    return from_cuda(launch_act_quant_swiglu(gate, up, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes,
+                                             scale_x, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status_t bitnet_hbitlinear_forward_swiglu(const void *gate, const void *up, bitnet_dtype_t xdt, int64_t M,
+                                                 int64_t K, const float *gain, float eps, int fwht,
+                                                 bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
+                                                 int64_t N, float *out, void *ws, size_t ws_bytes, void *stream) {
+    if (M > 0 && (!up || !aligned16(up))) {
+        // validate the rest first so that shape errors keep their own status
+        const bitnet_status_t st = validate_act(gate, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
+        return st != BITNET_OK ? st : BITNET_ERR_INVALID_ARG;
+    }
+    return forward_ws(gate, up, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, ws, ws_bytes, stream);
 }
 
 int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {

@@ -41,6 +41,10 @@ struct ZeroFill {
 cudaError_t launch_act_quant(const void *X, bool bf16, int64_t M, int K, const float *gain, float eps,
                              int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s,
                              ZeroFill zf = ZeroFill());
+// The same with the input formed as the SwiGLU product silu(gate) * up, elementwise.
+cudaError_t launch_act_quant_swiglu(const void *gate, const void *up, bool bf16, int64_t M, int K, const float *gain,
+                                    float eps, int fwht, int mode, int8_t *codes, float *scale_x, cudaStream_t s,
+                                    ZeroFill zf = ZeroFill());
 
 size_t pack_workspace_bytes();
 cudaError_t launch_pack(const float *W, int64_t N, int64_t K, float eps, uint8_t *packed, float *alpha,
@@ -76,10 +80,12 @@ double gemm_tile_cost(int bt, int splits, int M, int N, int K, int sms);
 bool gemm_force_tile(int bt);
 
 // The forward's kernels (act_quant, then GEMV or GEMM), arguments validated;
-// tile_cnt points at kSplitCounters ints of workspace for a split-K GEMM.
+// tile_cnt points at kSplitCounters ints of workspace for a split-K GEMM.  With
+// `up` given, X is the SwiGLU gate and the input is silu(X) * up.
 cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
                             int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
-                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s);
+                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
+                            const void *up = nullptr);
 
 // Launch the timeout self-test kernel.
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);

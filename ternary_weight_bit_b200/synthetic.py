@@ -46,13 +46,15 @@ def outlier_channels(K: int, count: int, gen: torch.Generator) -> torch.Tensor:
 
 @dataclass
 class Case:
-    """One H-BitLinear problem: activations X [M, K] and latent weights W [N, K]."""
+    """One H-BitLinear problem: activations X [M, K] and latent weights W [N, K].
+    With `up` set, X is the SwiGLU gate and the layer's input is silu(X) * up."""
     name: str
     X: torch.Tensor          # float32 (or bfloat16 when x_dtype == "bf16")
     W: torch.Tensor          # float32 [N, K]
     fwht: bool
     mode: str                # "int8" or "int4"
     eps: float = 1e-5
+    up: torch.Tensor | None = None
 
     @property
     def M(self) -> int:
@@ -70,12 +72,17 @@ class Case:
 def make_case(name: str, M: int, K: int, N: int, *, x_kind: str = "normal", outliers: int = 0,
               outlier_gain: float = 20.0, x_dtype: str = "f32", w_std: float = 0.02,
               fwht: bool = True, mode: str = "int8", seed: int = 0) -> Case:
-    """Draw X, the outlier permutation, then W, from one generator seeded ``seed``."""
+    """Draw X (for x_kind "swiglu": the gate, then up), the outlier permutation, then W,
+    from one generator seeded ``seed``."""
     gen = generator(seed)
+    up = None
     if x_kind == "normal":
         X = gaussian((M, K), 1.0, gen)
     elif x_kind == "student_t3":
         X = student_t3((M, K), gen)
+    elif x_kind == "swiglu":
+        X = gaussian((M, K), 2.0, gen)   # gate pre-activations
+        up = gaussian((M, K), 1.0, gen)
     else:
         raise ValueError(f"unknown x_kind {x_kind!r}")
     if outliers:
@@ -84,9 +91,10 @@ def make_case(name: str, M: int, K: int, N: int, *, x_kind: str = "normal", outl
     W = gaussian((N, K), w_std, gen)
     if x_dtype == "bf16":
         X = X.to(torch.bfloat16)
+        up = None if up is None else up.to(torch.bfloat16)
     elif x_dtype != "f32":
         raise ValueError(f"unknown x_dtype {x_dtype!r}")
-    return Case(name, X, W, fwht, mode)
+    return Case(name, X, W, fwht, mode, up=up)
 
 
 # --------------------------------------------------------------------------- workloads
@@ -105,6 +113,11 @@ def wdown_int4(M: int = 2048, K: int = 8192, N: int = 2048, seed: int = 0) -> Ca
     """Wdown-style H-BitLinear, int4 absmean + FWHT: Student-t(3) X with 1% channels x50."""
     return make_case(f"wdown_int4_M{M}_N{N}_K{K}", M, K, N, x_kind="student_t3",
                      outliers=round(0.01 * K), outlier_gain=50.0, fwht=True, mode="int4", seed=seed)
+
+
+def wdown_swiglu(M: int = 2048, K: int = 8192, N: int = 2048, seed: int = 0) -> Case:
+    """The FFN down projection on its SwiGLU input: gate N(0, 2^2), up N(0, 1) [M, K]; int4 + FWHT."""
+    return make_case(f"wdown_swiglu_M{M}_N{N}_K{K}", M, K, N, x_kind="swiglu", fwht=True, mode="int4", seed=seed)
 
 
 def prefill_int8(M: int = 4096, K: int = 4096, N: int = 4096, fwht: bool = False, seed: int = 0) -> Case:

@@ -289,6 +289,50 @@ def test_forward_split_k_forced_tiles(tile):
         tb.bitnet_gemm_force_token_tile(0)
 
 
+def _swiglu_case(M, K, N, mode, fwht, xdt, seed, sample_rows=None):
+    gen = torch.Generator().manual_seed(seed)
+    gate = torch.randn(M, K, generator=gen) * 2.0
+    up = torch.randn(M, K, generator=gen)
+    W = torch.randn(N, K, generator=gen) * 0.02
+    if xdt == "bf16":
+        gate, up = gate.to(torch.bfloat16), up.to(torch.bfloat16)
+    gd, ud = gate.to(DEV), up.to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(W.to(DEV))
+    out = tb.bitnet_hbitlinear_forward_swiglu(gd, ud, packed, alpha, N, fwht=fwht, mode=mode)
+    codes, gscale = tb.bitnet_act_quant_swiglu(gd, ud, fwht=fwht, mode=mode)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if sample_rows is None else sample_rows
+    g32, u32 = gate.float().numpy()[rows], up.float().numpy()[rows]
+    p_ref, a_ref, _ = ref.pack_weights(W.numpy())
+    m = MODES[mode]
+    r = ref.hbitlinear_forward(ref.swiglu(g32, u32), p_ref, a_ref, N, fwht_on=fwht, mode=m)
+    sh = ref.shadow_swiglu(g32, u32, eps=1e-5, fwht_on=fwht, mode=m)
+    gcodes, gs, gout = host(codes)[rows], host(gscale)[rows], host(out)[rows]
+    label = f"swiglu M={M} K={K} N={N} {mode} fwht={fwht} {xdt}"
+    parity.check_codes(gcodes, r.codes, sh, label)
+    parity.check_scale_bound(gs, r.scale_x, K, m, label)
+    parity.check_out_same_codes(gout, ref.dequant(ref.gemm_packed(gcodes, p_ref, N), gs, a_ref, m), label)
+    parity.check_out_end_to_end(gout, r.out, gcodes, r.codes, r.scale_x, a_ref, m, label)
+    assert tb.bitnet_get_last_device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,N,mode,fwht,xdt", [
+    (1, 2048, 512, "int4", True, "f32"),     # decode kernel
+    (8, 8192, 2048, "int4", True, "f32"),    # decode kernel, Wdown-like
+    (13, 1024, 700, "int8", False, "bf16"),  # decode kernel, ragged N, plain quantiser
+    (300, 4096, 1000, "int4", True, "f32"),  # tcgen05 kernel, ragged
+    (129, 2048, 640, "int8", True, "bf16"),
+])
+def test_forward_swiglu(M, K, N, mode, fwht, xdt):
+    # silu(gate) * up formed inside the activation kernel (BitNetV2FFN.forward's down projection)
+    _swiglu_case(M, K, N, mode, fwht, xdt, seed=M * 31 + K)
+
+
+def test_forward_swiglu_wdown_full_size_sampled():
+    # the Wdown-style shape: intermediate 8192 -> 2048, int4 + FWHT, 2048 tokens
+    _swiglu_case(2048, 8192, 2048, "int4", True, "f32", seed=3, sample_rows=_sample(2048, 24))
+
+
 def _sample(M, n=32, seed=0):
     rng = np.random.default_rng(seed)
     rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, n - 2, replace=False)]))
