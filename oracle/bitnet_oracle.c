@@ -368,3 +368,76 @@ int oracle_dequant(const int32_t *acc, const float *scale_x, float alpha, int mo
     }
     return ORACLE_OK;
 }
+
+/* ---------------------------------------------------------------------------
+ * Low-bit KV cache (NEXT row f3).  [v2] BitNetV2Attention._quantize_kv_head with
+ * ActQuantINT8STE / ActQuantINT4STE: per row of D values of a [B, H, S, D] key or
+ * value tensor (rows ordered (b, h, s)):
+ *   token s = 0 (the BOS token) always int8 absmax:
+ *       scale = max|x| + eps;  code = clamp(rne((127 / scale) * x), -128, 127);
+ *       step = scale / 127
+ *   tokens s >= 1 with bits = 4: int4 absmean:
+ *       scale = mean|x| + eps; code = clamp(rne((sqrt7 / scale) * x), -8, 7);
+ *       step = scale / sqrt7
+ *   tokens s >= 1 with bits = 3:
+ *       scale = max|x| + eps;  code = clamp(rne((3 / scale) * x), -4, 3);
+ *       step = scale / 3
+ *   tokens s >= 1 with bits = 8: as the BOS token.
+ * The page returns the fake-quantised values step * code; deq (if not NULL) gets
+ * them, codes and step are the stored form.  mean|x| is summed sequentially.
+ * ------------------------------------------------------------------------- */
+int oracle_kv_quant(const float *kv, int64_t BH, int64_t S, int64_t D, int bits, float eps,
+                    int8_t *codes, float *step, float *deq)
+{
+    if (BH < 0 || S < 0 || D <= 0) return ORACLE_BAD_ARG;
+    if (bits != 3 && bits != 4 && bits != 8) return ORACLE_BAD_ARG;
+    for (int64_t r = 0; r < BH * S; ++r) {
+        const float *x = kv + r * D;
+        const int rbits = (r % S == 0) ? 8 : bits;
+        float stat = 0.0f, Q, lo, hi;
+        if (rbits == 4) {
+            float sum = 0.0f;
+            for (int64_t k = 0; k < D; ++k) sum += fabsf(x[k]);
+            stat = sum / (float)D;
+            Q = q_int4(); lo = -8.0f, hi = 7.0f;
+        } else {
+            for (int64_t k = 0; k < D; ++k) stat = fabsf(x[k]) > stat ? fabsf(x[k]) : stat;
+            if (rbits == 8) { Q = q_int8(); lo = -128.0f; hi = 127.0f; }
+            else { Q = 3.0f; lo = -4.0f; hi = 3.0f; }
+        }
+        float scale = stat + eps;
+        float s = Q / scale;
+        float st = scale / Q;
+        step[r] = st;
+        for (int64_t k = 0; k < D; ++k) {
+            float c = clampf(rne(s * x[k]), lo, hi);
+            codes[r * D + k] = (int8_t)c;
+            if (deq) deq[r * D + k] = st * c;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* fp64 pre-rounding value s * x of every KV code (see oracle_shadow_prerounding). */
+int oracle_shadow_kv(const float *kv, int64_t BH, int64_t S, int64_t D, int bits, double eps, double *v)
+{
+    if (BH < 0 || S < 0 || D <= 0) return ORACLE_BAD_ARG;
+    if (bits != 3 && bits != 4 && bits != 8) return ORACLE_BAD_ARG;
+    for (int64_t r = 0; r < BH * S; ++r) {
+        const float *x = kv + r * D;
+        const int rbits = (r % S == 0) ? 8 : bits;
+        double stat = 0.0, Q;
+        if (rbits == 4) {
+            for (int64_t k = 0; k < D; ++k) stat += fabs((double)x[k]);
+            stat /= (double)D;
+            Q = sqrt(7.0);
+        } else {
+            for (int64_t k = 0; k < D; ++k) stat = fabs((double)x[k]) > stat ? fabs((double)x[k]) : stat;
+            Q = rbits == 8 ? 127.0 : 3.0;
+        }
+        const double s = Q / (stat + eps);
+        for (int64_t k = 0; k < D; ++k) v[r * D + k] = s * (double)x[k];
+    }
+    return ORACLE_OK;
+}
+

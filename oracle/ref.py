@@ -52,10 +52,13 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_gemm_packed.argtypes = [P, P, I64, I64, I64, P]
     L.oracle_dequant.argtypes = [P, P, F, I, I64, I64, P]
     L.oracle_swiglu.argtypes = [P, P, I64, P]
+    L.oracle_kv_quant.argtypes = [P, I64, I64, I64, I, F, P, P, P]
+    L.oracle_shadow_kv.argtypes = [P, I64, I64, I64, I, D, P]
     L.oracle_shadow_swiglu.argtypes = [P, P, I64, I64, P, D, I, I, P]
     for name in ("oracle_rmsnorm", "oracle_fwht", "oracle_act_quant", "oracle_shadow_prerounding",
                  "oracle_ternarize", "oracle_pack", "oracle_unpack", "oracle_gemm_int",
-                 "oracle_gemm_packed", "oracle_dequant", "oracle_swiglu", "oracle_shadow_swiglu"):
+                 "oracle_gemm_packed", "oracle_dequant", "oracle_swiglu", "oracle_shadow_swiglu",
+                 "oracle_kv_quant", "oracle_shadow_kv"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -152,6 +155,29 @@ def shadow_swiglu(gate, up, g=None, eps: float = 1e-5, fwht_on: bool = False, mo
     gp = None if g is None else _f32(g)
     _check("shadow_swiglu", L.oracle_shadow_swiglu(_p(ga), _p(u), M, K, None if gp is None else _p(gp),
                                                    float(np.float32(eps)), int(fwht_on), mode, _p(v)))
+    return v
+
+
+def kv_quant(kv, bits: int, eps: float = 1e-5, L=None):
+    """Low-bit KV cache of a [B, H, S, D] (or [BH, S, D]) tensor: (codes int8, step fp32 [.., S], deq fp32)."""
+    L = L or lib()
+    x = _f32(kv)
+    S, D = x.shape[-2], x.shape[-1]
+    BH = x.size // (S * D) if S * D else 0
+    codes = np.empty(x.shape, dtype=np.int8)
+    step = np.empty(x.shape[:-1], dtype=np.float32)
+    deq = np.empty(x.shape, dtype=np.float32)
+    _check("kv_quant", L.oracle_kv_quant(_p(x), BH, S, D, bits, eps, _p(codes), _p(step), _p(deq)))
+    return codes, step, deq
+
+
+def shadow_kv(kv, bits: int, eps: float = 1e-5, L=None) -> np.ndarray:
+    L = L or lib()
+    x = _f32(kv)
+    S, D = x.shape[-2], x.shape[-1]
+    BH = x.size // (S * D) if S * D else 0
+    v = np.empty(x.shape, dtype=np.float64)
+    _check("shadow_kv", L.oracle_shadow_kv(_p(x), BH, S, D, bits, float(np.float32(eps)), _p(v)))
     return v
 
 

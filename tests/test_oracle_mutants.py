@@ -36,6 +36,11 @@ MUTANTS = {
     "swiglu_sigmoid_only": ("float silu = gv / den;", "float silu = 1.0f / den;"),
     "swiglu_wrong_exp_sign": ("float den = 1.0f + expf(-gv);", "float den = 1.0f + expf(gv);"),
     "swiglu_drops_up": ("out[i] = silu * up[i];", "out[i] = silu;"),
+    "kv_bos_not_int8": ("const int rbits = (r % S == 0) ? 8 : bits;\n        float stat",
+                        "const int rbits = bits;\n        float stat"),
+    "kv_3bit_q_is_4": ("else { Q = 3.0f; lo = -4.0f; hi = 3.0f; }", "else { Q = 4.0f; lo = -4.0f; hi = 3.0f; }"),
+    "kv_step_without_eps": ("float scale = stat + eps;\n        float s = Q / scale;",
+                            "float scale = stat;\n        float s = Q / (stat + eps);"),
 }
 
 

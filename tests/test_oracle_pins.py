@@ -332,3 +332,72 @@ def test_shadow_swiglu_agrees_with_fp32_codes_away_from_ties():
         want = np.clip(np.rint(v), lo, hi)
         far = np.abs(v - np.floor(v) - 0.5) > 1e-3
         np.testing.assert_array_equal(q[far], want[far])
+
+
+# ----------------------------------------------------------------------------- low-bit KV cache
+# (bitnet_v2_engine.py page, BitNetV2Attention._quantize_kv_head)
+def test_kv_hand_case():
+    # one head, two tokens of D = 4: x = [1, -2, 0.5, 3]; computed by hand from the page's formulas
+    x = np.array([[[1.0, -2.0, 0.5, 3.0], [1.0, -2.0, 0.5, 3.0]]], np.float32)
+    c3, s3, d3 = ref.kv_quant(x, 3)
+    c4, s4, _ = ref.kv_quant(x, 4)
+    # BOS token: int8 absmax, 127 / (3 + 1e-5) * x -> [42.33, -84.67, 21.17, 127.0]
+    assert c3[0, 0].tolist() == [42, -85, 21, 127] == c4[0, 0].tolist()
+    assert _ulp_rel(s3[0, 0], (3.0 + 1e-5) / 127.0) < 3e-7
+    # 3-bit: 3 / (3 + 1e-5) * x -> [0.99999, -1.99999, 0.499998, 2.99999]
+    assert c3[0, 1].tolist() == [1, -2, 0, 3]
+    assert _ulp_rel(s3[0, 1], (3.0 + 1e-5) / 3.0) < 3e-7
+    np.testing.assert_allclose(d3[0, 1], np.array([1, -2, 0, 3]) * (3.0 + 1e-5) / 3.0, rtol=3e-7)
+    # 4-bit absmean: beta = 6.5 / 4 = 1.625, sqrt7 / (1.625 + 1e-5) * x -> [1.63, -3.26, 0.81, 4.88]
+    assert c4[0, 1].tolist() == [2, -3, 1, 5]
+    assert _ulp_rel(s4[0, 1], (1.625 + 1e-5) / math.sqrt(7.0)) < 3e-7
+
+
+def test_kv_3bit_tie_table():
+    # eps = 0 and gamma = 6: the multiplier 3 / 6 = 0.5 is exact, so 0.5 * x lands on half-integers
+    x = np.array([[[6.0, 1.0, 3.0, 5.0, -1.0, -3.0, -5.0, -6.0]] * 2], np.float32)
+    codes, step, deq = ref.kv_quant(x, 3, eps=0.0)
+    assert codes[0, 1].tolist() == [3, 0, 2, 2, 0, -2, -2, -3]  # round half to even
+    assert step[0, 1] == 2.0
+    np.testing.assert_array_equal(deq[0, 1], 2.0 * codes[0, 1])
+
+
+def test_kv_absmax_codes_stay_inside_the_symmetric_range():
+    # |x| <= gamma makes |3x / (gamma + eps)| < 3.5 and |127x / (gamma + eps)| < 127.5: -4 and -128 never occur
+    kv = np.random.default_rng(11).standard_t(3, size=(4, 2, 64, 128)).astype(np.float32)
+    for bits, lim in ((3, 3), (8, 127)):
+        codes, _, _ = ref.kv_quant(kv, bits)
+        rest = codes[..., 1:, :]  # token 0 is always int8
+        assert rest.min() >= -lim and rest.max() <= lim
+        assert (np.abs(rest).max(axis=-1) == lim).all()  # the max element reaches the top code
+        assert np.abs(codes[..., 0, :]).max() <= 127
+
+
+def test_kv_reconstruction_within_half_a_step():
+    kv = np.random.default_rng(12).normal(size=(2, 3, 17, 64)).astype(np.float32)
+    for bits in (3, 8):
+        _, step, deq = ref.kv_quant(kv, bits)
+        err = np.abs(deq.astype(np.float64) - kv)
+        assert (err <= 0.5 * step[..., None] * (1 + 1e-5) + 1e-7).all()
+
+
+def test_kv_bos_token_is_always_int8():
+    kv = np.random.default_rng(13).normal(size=(3, 5, 9, 32)).astype(np.float32)
+    c8, s8, _ = ref.kv_quant(kv, 8)
+    for bits in (3, 4):
+        c, s, _ = ref.kv_quant(kv, bits)
+        np.testing.assert_array_equal(c[:, :, 0], c8[:, :, 0])
+        np.testing.assert_array_equal(s[:, :, 0], s8[:, :, 0])
+        assert np.abs(c[:, :, 1:]).max() <= (3 if bits == 3 else 8)
+
+
+def test_kv_shadow_agrees_away_from_ties():
+    kv = np.random.default_rng(14).normal(size=(2, 4, 33, 64)).astype(np.float32)
+    for bits, lo, hi in ((3, -4, 3), (4, -8, 7), (8, -128, 127)):
+        codes, _, _ = ref.kv_quant(kv, bits)
+        v = ref.shadow_kv(kv, bits)
+        lo_b = np.where(np.arange(33)[None, None, :, None] == 0, -128, lo)
+        hi_b = np.where(np.arange(33)[None, None, :, None] == 0, 127, hi)
+        want = np.clip(np.rint(v), lo_b, hi_b)
+        far = np.abs(v - np.floor(v) - 0.5) > 1e-3
+        np.testing.assert_array_equal(codes[far], want[far])
