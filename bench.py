@@ -502,9 +502,229 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+# ----------------------------------------------------------------------------- KV-cache workload
+KV_SHAPE = (1, 32, 4096, 128)  # B, H, S, D: one layer's keys (and values) over a 4096-token context
+KV_BITS = 4
+KV_TEXT = ("low-bit KV cache (BitNetV2Attention._quantize_kv_head): K and V [1, 32, 4096, 128] fp32, Student-t(3) "
+           "with every 16th channel x6; token 0 int8, the rest int4 absmean; codes int8 + per-row step")
+
+
+def kv_inputs(seed=0):
+    from ternary_weight_bit_b200 import synthetic
+    gen = synthetic.generator(seed)
+    out = []
+    for _ in range(2):  # K, then V
+        t = synthetic.student_t3(KV_SHAPE, gen)
+        t[..., ::16] *= 6.0
+        out.append(t)
+    return out
+
+
+def time_oracle_kv(budget_s: float, steps: int | None = None):
+    """The oracle kv_quant on a sample of heads, extrapolated to all heads of K and V."""
+    import numpy as np
+    from oracle import ref
+    K, V = kv_inputs()
+    B, H, S, D = KV_SHAPE
+    heads = 1
+    totals = []
+    t_begin = time.perf_counter()
+    while True:
+        t = 0.0
+        for T in (K, V):
+            x = np.ascontiguousarray(T[:, :heads].numpy())
+            t0 = time.perf_counter()
+            ref.kv_quant(x, KV_BITS)
+            t += (time.perf_counter() - t0) * (H / heads)
+        totals.append(t)
+        if steps is not None and len(totals) >= steps:
+            break
+        if steps is None and (time.perf_counter() - t_begin >= budget_s or len(totals) >= 50):
+            break
+    per_step = statistics.median(totals)
+    desc = (f"oracle (single-threaded C) kv_quant on {heads} of {H} heads of K and V, extrapolated to all heads; "
+            f"{len(totals)} step(s), median")
+    return B * S / per_step, desc, per_step
+
+
+def run_kv(args):
+    import torch
+    import ternary_weight_bit_b200 as tb
+
+    world, rank, local = dist_setup(args.gpus)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    host = kv_inputs()
+    B, H, S, D = KV_SHAPE
+    in_bytes = sum(t.numel() * 4 for t in host)
+    R = max(2, math.ceil(4 * l2 / in_bytes))
+    rot = []
+    for r in range(R):
+        rot.append([(t.to(dev), torch.empty(KV_SHAPE, dtype=torch.int8, device=dev),
+                     torch.empty(KV_SHAPE[:-1], dtype=torch.float32, device=dev)) for t in host])
+    torch.cuda.synchronize()
+
+    def step(r):
+        for x, codes, st in rot[r]:
+            tb.bitnet_kv_quant(x, bits=KV_BITS, codes=codes, step=st)
+
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for i in range(max(1, min(args.warmup, R))):
+            step(i % R)
+    stream.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+    stream.synchronize()
+    gpu_uuid = ""
+    try:
+        gpu_uuid = "GPU-" + str(props.uuid) if not str(props.uuid).startswith("GPU-") else str(props.uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            graphs[i % R].replay()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    elapsed = e0.elapsed_time(e1)
+    max_ms, tokens_all = aggregate(elapsed, args.steps * B * S, world, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    status = tb.bitnet_get_last_device_status(stream)
+    # the kernel alone: one graph over every rotation, replayed, so that graph-launch
+    # gaps between steps do not count against the launch duration
+    gg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gg, stream=stream):
+        for r in range(R):
+            step(r)
+    reps = max(3, min(200, int(400 / R)))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            gg.replay()
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            gg.replay()
+    k1.record(stream)
+    k1.synchronize()
+    launches = reps * R * 2  # two launches (K, V) per step
+    avg_launch_s = k0.elapsed_time(k1) / 1e3 / launches
+    bytes_per_launch = B * H * S * (4 * D + D + 4)  # read fp32, write int8 codes and the fp32 step
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = bytes_per_launch / avg_launch_s / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": profile_traffic("kv_quant_traffic_kvcache", "kv_quant.cu"),
+            "kernel": "kv_quant_kernel (a warp per group of (b, h, s) rows, 16-byte loads, shuffle reductions)",
+            "peak_source": f"hbm_gbs of {peak_src} MEASURED_PEAKS.json (copy, burst)",
+            "avg_launch_us": round(avg_launch_s * 1e6, 3), "bytes_per_launch": bytes_per_launch}
+    # end to end through the public API: H2D of K and V, quantise, D2H of codes and steps
+    pin_in = [t.pin_memory() for t in host]
+    pin_c = [torch.empty(KV_SHAPE, dtype=torch.int8).pin_memory() for _ in host]
+    pin_s = [torch.empty(KV_SHAPE[:-1], dtype=torch.float32).pin_memory() for _ in host]
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_once(r):
+        for hi, hc, hs, (x, codes, st) in zip(pin_in, pin_c, pin_s, rot[r]):
+            x.copy_(hi, non_blocking=True)
+            tb.bitnet_kv_quant(x, bits=KV_BITS, codes=codes, step=st)
+            hc.copy_(codes, non_blocking=True)
+            hs.copy_(st, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_once(0)
+    stream.synchronize()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps):
+            e2e_once(i % R)
+    x1.record(stream)
+    x1.synchronize()
+    e2e_max, e2e_tokens = aggregate(x0.elapsed_time(x1), e2e_steps * B * S, world, dev)
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(tokens_all / (max_ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": KV_TEXT, "name": "kvcache",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"inputs rotate over {R} copies ({R * in_bytes / 2**20:.0f} MiB > 4x L2)",
+                       "cuda_graphs": True, "pdl": True},
+            "roofline": roof,
+            "e2e": {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": sum(c.numel() + 4 * s.numel()
+                                                                               for c, s in zip(pin_c, pin_s)),
+                    "note": "eager bitnet_kv_quant calls with pinned host K, V in and codes, steps out per step"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "device_status": status,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        graphs.clear()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, desc, _ = time_oracle_kv(budget_s=args.cpu_budget)
+            result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                      "sample": desc}
+        print(json.dumps(result), flush=True)
+
+
 def run_reference(args):
     world, rank, _ = dist_setup(args.gpus)
     if rank != 0:
+        return
+    if args.workload == "kvcache":
+        budget = max(10.0, min(150.0, 6.0 * (args.steps + args.warmup)))
+        if args.warmup:
+            time_oracle_kv(budget, steps=1)
+        v, desc, per_step = time_oracle_kv(budget, steps=args.steps)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": KV_TEXT, "name": "kvcache"},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
         return
     cases = workload_cases(args.workload)
     budget = max(10.0, min(150.0, 6.0 * (args.steps + args.warmup)))
@@ -532,7 +752,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    help="decode (default) | prefill | wdown | msweep_M<M>")
+                    help="decode (default) | prefill | wdown | wdown_swiglu | msweep_M<M> | kvcache")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -540,6 +760,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "kvcache":
+        run_kv(args)
     else:
         run_ours(args)
 

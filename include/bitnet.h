@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 3
+#define BITNET_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -220,6 +220,30 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
                                                               bitnet_act_mode_t mode, const uint8_t *packed,
                                                               const float *alpha, int64_t N, float *out,
                                                               void *stream);
+
+/* --------------------------------------------------------------------------
+ * bitnet_kv_quant -- the low-bit KV cache of a BitNet v2 attention layer.
+ * Definition: bitnet_v2_engine.py page, BitNetV2Attention._quantize_kv_head with
+ * quantize_act_int8 / quantize_act_int4 (Eq. 5/6).  Per row of D values of a
+ * post-RoPE key or value tensor [B][H][S][D] (passed as BH = B*H rows of S tokens):
+ *   token s = 0 (BOS, kept at 8 bits):  scale = max|x| + eps,  Q = 127, codes in [-128, 127]
+ *   tokens s >= 1, bits = 4:            scale = mean|x| + eps, Q = sqrt7, codes in [-8, 7]
+ *   tokens s >= 1, bits = 3:            scale = max|x| + eps,  Q = 3,  codes in [-4, 3]
+ *   tokens s >= 1, bits = 8:            as token 0
+ *   code = RoundClip(rne((Q / scale) * x)),  step = scale / Q,
+ * each an fp32 IEEE operation; step * code is the page's fake-quantised value.
+ *   kv     [BH][S][D] fp32 or bf16 (xdt), device, read only.
+ *   codes  [BH][S][D] int8, device, written (one code per byte).
+ *   step   [BH][S] fp32, device, written.
+ *   deq    [BH][S][D] fp32 or NULL: step * code.
+ * D must be a multiple of 4 and at most 1024 (BITNET_ERR_UNSUPPORTED_SHAPE);
+ * bits other than 3, 4, 8 are BITNET_ERR_INVALID_ARG.  The max of the 3- and 8-bit
+ * rows is exact; the mean of the 4-bit rows is summed in another order than a
+ * sequential loop, so a 4-bit code may differ by one at a rounding near-tie.
+ * ------------------------------------------------------------------------ */
+BITNET_API bitnet_status_t bitnet_kv_quant(const void *kv, bitnet_dtype_t xdt, int64_t BH, int64_t S, int64_t D,
+                                           int bits, float eps, int8_t *codes, float *step, float *deq,
+                                           void *stream);
 
 /* --------------------------------------------------------------------------
  * Prefill GEMM tile control (no counterpart on the pages).

@@ -26,7 +26,7 @@ __all__ = [
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
     "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_forward_gemm_plan",
-    "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu",
+    "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu", "bitnet_kv_quant",
 ]
 
 _MODES = {"int8": _native.ACT_INT8_ABSMAX, "int4": _native.ACT_INT4_ABSMEAN}
@@ -183,6 +183,27 @@ def bitnet_hbitlinear_forward_swiglu(gate: torch.Tensor, up: torch.Tensor, packe
                                                      int(bool(fwht)), mode_id(mode), _ptr(packed), _ptr(alpha), N,
                                                      _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def bitnet_kv_quant(kv: torch.Tensor, bits: int = 4, eps: float = 1e-5, dequant: bool = False, codes=None,
+                    step=None, deq=None, stream=None):
+    """Low-bit KV cache of a [..., S, D] key or value tensor (token 0 kept at int8).
+    Returns (codes int8 [..., S, D], step fp32 [..., S], deq fp32 [..., S, D] or None)."""
+    L = _native.load()
+    _need(kv, "kv")
+    S, D = kv.shape[-2], kv.shape[-1]
+    BH = kv.numel() // (S * D) if S * D else 0
+    codes = torch.empty(kv.shape, dtype=torch.int8, device=kv.device) if codes is None else codes
+    step = torch.empty(kv.shape[:-1], dtype=torch.float32, device=kv.device) if step is None else step
+    if dequant and deq is None:
+        deq = torch.empty(kv.shape, dtype=torch.float32, device=kv.device)
+    _need(codes, "codes", torch.int8, tuple(kv.shape))
+    _need(step, "step", torch.float32, tuple(kv.shape[:-1]))
+    if deq is not None:
+        _need(deq, "deq", torch.float32, tuple(kv.shape))
+    _native.check("bitnet_kv_quant", L.bitnet_kv_quant(_ptr(kv), _xdt(kv), BH, S, D, bits, eps, _ptr(codes),
+                                                       _ptr(step), _ptr(deq), _stream(stream)))
+    return codes, step, deq
 
 
 def bitnet_ternary_gemm(codes: torch.Tensor, scale_x: torch.Tensor, mode, packed: torch.Tensor,

@@ -317,6 +317,21 @@ bitnet_status_t bitnet_gemm_force_token_tile(int token_tile) {
     return gemm_force_tile(token_tile) ? BITNET_OK : BITNET_ERR_INVALID_ARG;
 }
 
+bitnet_status_t bitnet_kv_quant(const void *kv, bitnet_dtype_t xdt, int64_t BH, int64_t S, int64_t D, int bits,
+                                float eps, int8_t *codes, float *step, float *deq, void *stream) {
+    if (xdt != BITNET_F32 && xdt != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+    if (bits != 3 && bits != 4 && bits != 8) return BITNET_ERR_INVALID_ARG;
+    if (BH < 0 || S < 0 || BH > kMaxRows || S > kMaxRows || (S > 0 && BH > kMaxRows / S))
+        return BITNET_ERR_INVALID_ARG;
+    if (D < 4 || D > 1024 || D % 4 != 0) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    if (BH == 0 || S == 0) return BITNET_OK;
+    if (!kv || !codes || !step || !aligned16(kv) || !aligned16(codes) || !aligned16(step) ||
+        (deq && !aligned16(deq)))
+        return BITNET_ERR_INVALID_ARG;
+    return from_cuda(launch_kv_quant(kv, xdt == BITNET_BF16, BH, S, (int)D, bits, eps, codes, step, deq,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 bitnet_status_t bitnet_get_last_device_status(void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;

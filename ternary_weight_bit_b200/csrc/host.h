@@ -87,6 +87,11 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
                             int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
                             const void *up = nullptr);
 
+// Low-bit KV cache: kv [BH][S][D] (fp32 or bf16), D % 4 == 0, D <= 1024; bits 3, 4 or 8
+// for tokens s >= 1 (token 0 is always int8).  deq may be null.
+cudaError_t launch_kv_quant(const void *kv, bool bf16, int64_t BH, int64_t S, int D, int bits, float eps,
+                            int8_t *codes, float *step, float *deq, cudaStream_t s);
+
 // Launch the timeout self-test kernel.
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);
 

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 3
+    assert L.bitnet_abi_version() == 4
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
@@ -51,6 +51,19 @@ def test_gemm_token_tile_host_logic(L):
             assert L.bitnet_gemm_token_tile(4096, 4096, 4096) == good  # a forced tile wins
     finally:
         assert L.bitnet_gemm_force_token_tile(0) == _native.OK
+
+
+def test_kv_quant_validation(L):
+    s = P(0)
+    ok = _native.OK
+    assert L.bitnet_kv_quant(FAKE, 0, 2, 3, 128, 5, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG   # bits
+    assert L.bitnet_kv_quant(FAKE, 2, 2, 3, 128, 4, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG   # dtype
+    assert L.bitnet_kv_quant(FAKE, 0, 2, 3, 130, 4, 1e-5, FAKE, FAKE, None, s) == _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_kv_quant(FAKE, 0, 2, 3, 2048, 4, 1e-5, FAKE, FAKE, None, s) == _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_kv_quant(FAKE, 0, -1, 3, 128, 4, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_kv_quant(None, 0, 0, 3, 128, 3, 1e-5, None, None, None, s) == ok   # empty: nothing to do
+    assert L.bitnet_kv_quant(None, 0, 2, 3, 128, 3, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_kv_quant(P(4100), 0, 2, 3, 128, 3, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG
 
 
 def test_workspace_sizes(L):

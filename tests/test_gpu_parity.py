@@ -333,6 +333,48 @@ def test_forward_swiglu_wdown_full_size_sampled():
     _swiglu_case(2048, 8192, 2048, "int4", True, "f32", seed=3, sample_rows=_sample(2048, 24))
 
 
+# ----------------------------------------------------------------------------- low-bit KV cache
+@pytest.mark.parametrize("B,H,S,D,bits,xdt", [
+    (1, 2, 9, 128, 4, "f32"),
+    (2, 3, 17, 64, 3, "f32"),
+    (1, 4, 33, 256, 8, "bf16"),
+    (1, 1, 1, 128, 4, "f32"),     # the BOS token alone
+    (2, 2, 5, 100, 4, "f32"),     # D not a multiple of 32
+    (1, 1, 7, 1024, 3, "bf16"),
+    (1, 2, 3, 4, 4, "f32"),       # D = 4
+    (2, 3, 3, 32, 4, "bf16"),     # eight lanes per row, BOS rows beside absmean rows in one warp
+    (3, 5, 70, 192, 3, "f32"),    # sixteen lanes per row, ragged last warp
+])
+def test_kv_quant(B, H, S, D, bits, xdt):
+    gen = torch.Generator().manual_seed(B * 100 + S * 7 + D)
+    kv = synthetic.student_t3((B, H, S, D), gen)
+    kv[..., :: max(1, D // 8)] *= 6.0  # a few large channels, as post-RoPE keys have
+    if xdt == "bf16":
+        kv = kv.to(torch.bfloat16)
+    codes, step, deq = tb.bitnet_kv_quant(kv.to(DEV), bits=bits, dequant=True)
+    codes2, step2, none = tb.bitnet_kv_quant(kv.to(DEV), bits=bits)
+    torch.cuda.synchronize()
+    assert none is None
+    gc, gs, gd = host(codes), host(step), host(deq)
+    np.testing.assert_array_equal(host(codes2), gc)
+    np.testing.assert_array_equal(host(step2), gs)
+    x32 = kv.float().numpy()
+    oc, os_, _ = ref.kv_quant(x32, bits)
+    sh = ref.shadow_kv(x32, bits)
+    label = f"kv B={B} H={H} S={S} D={D} bits={bits} {xdt}"
+    # the 8- and 3-bit rows (and every BOS row) use an exact max: identical codes and steps
+    exact_rows = np.ones(x32.shape[:-1], bool) if bits != 4 else (np.arange(S) == 0)[None, None, :].repeat(B, 0).repeat(H, 1)
+    np.testing.assert_array_equal(gc[exact_rows], oc[exact_rows], err_msg=label)
+    np.testing.assert_array_equal(gs[exact_rows], os_[exact_rows], err_msg=label)
+    if bits == 4 and S > 1:
+        parity.check_codes(gc[:, :, 1:], oc[:, :, 1:], sh[:, :, 1:], label)
+        rel = np.abs(gs[:, :, 1:].astype(np.float64) - os_[:, :, 1:]) / os_[:, :, 1:]
+        assert rel.max() <= (D + 32 + 8) * 2.0 ** -24 + 4 * 2.0 ** -24, label  # sum order only
+    # the dequantised values are step * code, one rounding
+    np.testing.assert_array_equal(gd, gs[..., None] * gc.astype(np.float32))
+    assert tb.bitnet_get_last_device_status() == 0
+
+
 def _sample(M, n=32, seed=0):
     rng = np.random.default_rng(seed)
     rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, n - 2, replace=False)]))
