@@ -35,6 +35,8 @@
  *   - alpha = mean|W| is summed in double in index order, rounded once to float.
  *   - The dequant epilogue is out = (float)acc * ((alpha * scale_x) / Q).
  *   - silu(g) = g / (1 + e^-g) in fp32 (the page calls F.silu = g * sigmoid(g)).
+ *   - A bf16 output is the fp32 output rounded once to bf16, to nearest, ties to
+ *     even (the pages name a bf16 output only as a storage option).
  */
 #include <math.h>
 #include <stdint.h>
@@ -365,6 +367,36 @@ int oracle_dequant(const int32_t *acc, const float *scale_x, float alpha, int mo
     for (int64_t m = 0; m < M; ++m) {
         float f = (alpha * scale_x[m]) / Q;
         for (int64_t n = 0; n < N; ++n) out[m * N + n] = (float)acc[m * N + n] * f;
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * bf16 output (NEXT row f4).  bf16 keeps the sign, the 8 exponent bits and the top
+ * 7 fraction bits of an fp32 value.  A finite x lies between two adjacent bf16
+ * values: lo, x with its low 16 bits cleared (toward zero), and hi, the next one
+ * away from zero.  The result is the nearer of the two; at the exact midpoint,
+ * the one whose last kept bit is 0.  Stepping past the largest finite bf16 gives
+ * infinity, as IEEE rounding to nearest does.  A NaN stays a NaN (its top
+ * fraction bit set, so that dropping the low bits cannot make it infinite).
+ * out holds the bf16 bit patterns.
+ * ------------------------------------------------------------------------- */
+int oracle_round_bf16(const float *x, int64_t count, uint16_t *out)
+{
+    if (count < 0) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < count; ++i) {
+        uint32_t u;
+        memcpy(&u, &x[i], sizeof u);
+        const uint32_t kept = u >> 16;       /* sign, exponent, 7 fraction bits */
+        const uint32_t dropped = u & 0xFFFFu; /* what the truncation loses */
+        if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0) {
+            out[i] = (uint16_t)(kept | 0x0040u); /* NaN: quiet, never infinity */
+            continue;
+        }
+        uint32_t r = kept;
+        if (dropped > 0x8000u) r = kept + 1;                         /* nearer to hi */
+        else if (dropped == 0x8000u && (kept & 1u)) r = kept + 1;    /* midpoint: to even */
+        out[i] = (uint16_t)r; /* kept + 1 carries into the exponent when it must */
     }
     return ORACLE_OK;
 }

@@ -55,6 +55,7 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_kv_quant.argtypes = [P, I64, I64, I64, I, F, P, P, P]
     L.oracle_shadow_kv.argtypes = [P, I64, I64, I64, I, D, P]
     L.oracle_shadow_swiglu.argtypes = [P, P, I64, I64, P, D, I, I, P]
+    L.oracle_round_bf16.argtypes = [P, I64, P]
     for name in ("oracle_rmsnorm", "oracle_fwht", "oracle_act_quant", "oracle_shadow_prerounding",
                  "oracle_ternarize", "oracle_pack", "oracle_unpack", "oracle_gemm_int",
                  "oracle_gemm_packed", "oracle_dequant", "oracle_swiglu", "oracle_shadow_swiglu",
@@ -247,6 +248,15 @@ def dequant(acc, scale_x, alpha, mode: int, L=None) -> np.ndarray:
     M, N = acc.shape
     out = np.empty((M, N), dtype=np.float32)
     _check("dequant", L.oracle_dequant(_p(acc), _p(s), float(alpha), mode, M, N, _p(out)))
+    return out
+
+
+def round_bf16(x, L=None) -> np.ndarray:
+    """bf16 bit patterns (uint16) of x rounded to nearest, ties to even."""
+    L = L or lib()
+    x = _f32(x)
+    out = np.empty(x.shape, dtype=np.uint16)
+    _check("round_bf16", L.oracle_round_bf16(_p(x), x.size, _p(out)))
     return out
 
 

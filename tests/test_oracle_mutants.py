@@ -41,6 +41,9 @@ MUTANTS = {
     "kv_3bit_q_is_4": ("else { Q = 3.0f; lo = -4.0f; hi = 3.0f; }", "else { Q = 4.0f; lo = -4.0f; hi = 3.0f; }"),
     "kv_step_without_eps": ("float scale = stat + eps;\n        float s = Q / scale;",
                             "float scale = stat;\n        float s = Q / (stat + eps);"),
+    "bf16_truncates": ("if (dropped > 0x8000u) r = kept + 1;", "if (0) r = kept + 1;"),
+    "bf16_ties_away": ("else if (dropped == 0x8000u && (kept & 1u)) r = kept + 1;",
+                       "else if (dropped == 0x8000u) r = kept + 1;"),
 }
 
 

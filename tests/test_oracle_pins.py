@@ -20,6 +20,7 @@ import os
 import numpy as np
 import pytest
 import scipy.linalg
+import torch
 
 from oracle import ref
 
@@ -401,3 +402,89 @@ def test_kv_shadow_agrees_away_from_ties():
         want = np.clip(np.rint(v), lo_b, hi_b)
         far = np.abs(v - np.floor(v) - 0.5) > 1e-3
         np.testing.assert_array_equal(codes[far], want[far])
+
+
+# ----------------------------------------------------------------------------- bf16 output
+# (the fp32 output rounded once to bf16, to nearest, ties to even)
+def _bits(x):
+    return np.array([x], np.float32).view(np.uint32)[0]
+
+
+def _from_bits32(u):
+    return np.array([u], np.uint32).view(np.float32)[0]
+
+
+def _bf16_value(b):
+    return np.asarray(b, np.uint32) << 16
+
+
+def test_bf16_hand_table():
+    e = 2.0 ** -8
+    cases = [
+        (1.0 + e, 0x3F80),               # midpoint between 1 and 1 + 2^-7: the even one, 1
+        (1.0 + 3 * e, 0x3F82),           # midpoint between 1 + 2^-7 and 1 + 2^-6: the even one
+        (1.0 + e + 2.0 ** -23, 0x3F81),  # just past the midpoint: up
+        (1.0 + e - 2.0 ** -23, 0x3F80),  # just short of it: down
+        (-(1.0 + 3 * e), 0xBF82),        # the sign is kept, the magnitude rounds alike
+        (3.5, 0x4060),                   # representable: unchanged
+        (0.0, 0x0000),
+        (-0.0, 0x8000),
+        (65280.0 + 128.0, 0x4780),       # 2^16 - 2^8 + 2^7: midpoint, odd neighbour 0x477F, even 0x4780
+    ]
+    got = ref.round_bf16(np.array([c[0] for c in cases], np.float32))
+    for (x, want), g in zip(cases, got):
+        assert int(g) == want, (x, hex(int(g)), hex(want))
+
+
+def test_bf16_special_bit_patterns():
+    pats = np.array([0x7F7FFFFF,   # largest fp32: past the largest bf16 -> infinity
+                     0x7F7F7FFF,   # just below that midpoint -> largest finite bf16
+                     0x7F800000,   # infinity stays
+                     0xFF800000,   # -infinity stays
+                     0x00000001,   # smallest subnormal -> +0
+                     0x00008000,   # subnormal midpoint, even neighbour 0
+                     0x00018000,   # subnormal midpoint, odd neighbour 1 -> 2
+                     0x7FC00000,   # quiet NaN
+                     0x7F800001],  # signalling NaN: must not become infinity
+                    np.uint32)
+    got = ref.round_bf16(pats.view(np.float32)).astype(np.uint32)
+    assert list(got[:7]) == [0x7F80, 0x7F7F, 0x7F80, 0xFF80, 0x0000, 0x0000, 0x0002]
+    for g in got[7:]:
+        assert (g & 0x7F80) == 0x7F80 and (g & 0x7F) != 0  # NaN
+
+
+def test_bf16_is_the_nearest_lattice_point_by_brute_force():
+    # every result is a bf16 value (a 16-bit pattern), no adjacent bf16 value is nearer,
+    # and a result at exactly half a bf16 step has an even last bit
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-60, 60, 20000))).astype(np.float32)
+    x[:2000] = (np.float32(1.0) + rng.integers(0, 2 ** 16, 2000).astype(np.float32) * np.float32(2.0 ** -23)) \
+        * np.where(rng.random(2000) < 0.5, -1, 1).astype(np.float32)  # dense near the midpoints of [1, 2)
+    b = ref.round_bf16(x).astype(np.uint32)
+    r = _bf16_value(b).view(np.float32).astype(np.float64)
+    x64 = x.astype(np.float64)
+    d = np.abs(x64 - r)
+    for nb in (b + 1, b - 1):
+        ok = (nb & 0x7F80) != 0x7F80  # skip neighbours that are not finite
+        rn = _bf16_value(nb).view(np.float32).astype(np.float64)
+        dn = np.abs(x64 - rn)
+        assert (d[ok] <= dn[ok]).all()
+        tie = ok & (d == dn)
+        assert ((b[tie] & 1) == 0).all()
+    assert (d <= np.abs(x64) * 2.0 ** -8 + 1e-300).all()  # half a step of 2^-7 relative at most
+
+
+def test_bf16_agrees_with_torch_cpu_conversion():
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal(50000) * np.exp2(rng.integers(-30, 30, 50000))).astype(np.float32)
+    t = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(ref.round_bf16(x), t)
+
+
+def test_bf16_is_odd_and_monotone():
+    rng = np.random.default_rng(23)
+    x = np.sort((rng.standard_normal(10000) * 100).astype(np.float32))
+    b = ref.round_bf16(x)
+    np.testing.assert_array_equal(ref.round_bf16(-x), b ^ np.uint16(0x8000))
+    v = _bf16_value(b.astype(np.uint32)).view(np.float32)
+    assert (np.diff(v) >= 0).all()
