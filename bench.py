@@ -95,11 +95,11 @@ def make_inputs(cases, seed=0):
     return out
 
 
-def algorithmic_bytes(M, N, K, xdt):
-    """Bytes the method must move per forward: X in, codes/scales round trip, packed W, fp32 out."""
+def algorithmic_bytes(M, N, K, xdt, out_bytes=4):
+    """Bytes the method must move per forward: X in, codes/scales round trip, packed W, fp32 (or bf16) out."""
     xb = 2 if xdt == "bf16" else 4
     act = M * K * xb + M * K + 4 * M            # act_quant: read X, write codes + scale
-    gemm = N * K // 4 + M * K + 4 * M + 4 * M * N + 4  # packed W, codes, scales, out, alpha
+    gemm = N * K // 4 + M * K + 4 * M + out_bytes * M * N + 4  # packed W, codes, scales, out, alpha
     return act, gemm
 
 
@@ -212,7 +212,7 @@ def aggregate(elapsed_ms: float, tokens: float, world: int, backend_device=None)
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
-def time_oracle(cases, budget_s: float, steps: int | None = None):
+def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool = False):
     """Time the oracle on a bounded sample of the workload.  Each case runs the full
     per-token act_quant and the integer GEMM on a sample of output columns; the
     time is extrapolated to all N columns.  Returns (tokens/s, description, steps)."""
@@ -243,7 +243,9 @@ def time_oracle(cases, budget_s: float, steps: int | None = None):
             q, s = ref.act_quant(X, None, c.eps, c.fwht, mode)
             t1 = time.perf_counter()
             acc = ref.gemm_packed(q, packed[:ncols], ncols)
-            ref.dequant(acc, s, alpha, mode)
+            o = ref.dequant(acc, s, alpha, mode)
+            if bf16_out:
+                ref.round_bf16(o)
             t2 = time.perf_counter()
             t_step += (t1 - t0) + (t2 - t1) * (c.N / ncols)
         totals.append(t_step)
@@ -276,6 +278,11 @@ def run_ours(args):
 
     cases = workload_cases(args.workload)
     host = make_inputs(cases)
+    bf16_out = args.out_dtype == "bf16"
+    if bf16_out and any(c.up is not None for c in host):
+        raise SystemExit("--out-dtype bf16 applies to the plain forward workloads")
+    out_dtype = torch.bfloat16 if bf16_out else torch.float32
+    out_bytes = 2 if bf16_out else 4
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
 
@@ -300,13 +307,16 @@ def run_ours(args):
             U = None if c.up is None else c.up.to(dev)
             ws = torch.empty((max(tb.bitnet_forward_workspace_bytes(c.M, c.K), 256),), dtype=torch.uint8,
                              device=dev)
-            out = torch.empty((c.M, c.N), dtype=torch.float32, device=dev)
+            out = torch.empty((c.M, c.N), dtype=out_dtype, device=dev)
             items.append((X, p.clone() if r else p, a, out, ws, U))
         rot.append(items)
     torch.cuda.synchronize()
 
     def forward(c, X, p, a, out, ws, U):
-        if U is None:
+        if U is None and bf16_out:
+            tb.bitnet_hbitlinear_forward_ex(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode,
+                                            out_dtype=torch.bfloat16, out=out, ws=ws)
+        elif U is None:
             tb.bitnet_hbitlinear_forward(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
         else:
             tb.bitnet_hbitlinear_forward_swiglu(X, U, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out,
@@ -381,7 +391,10 @@ def run_ours(args):
 
     def gemm_pass(r):
         for c, (codes, scale), (X, p, a, out, ws, U) in zip(host, codes_scales, rot[r]):
-            tb.bitnet_ternary_gemm(codes, scale, c.mode, p, a, c.N, out=out)
+            if bf16_out:
+                tb.bitnet_ternary_gemm_ex(codes, scale, c.mode, p, a, c.N, out_dtype=torch.bfloat16, out=out)
+            else:
+                tb.bitnet_ternary_gemm(codes, scale, c.mode, p, a, c.N, out=out)
 
     gg = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -404,7 +417,7 @@ def run_ours(args):
     k1.synchronize()
     gemm_ms = k0.elapsed_time(k1)
     launches = reps * R * len(host)
-    gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32")[1] for c in host)
+    gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32", out_bytes)[1] for c in host)
     gemm_ops = reps * R * sum(2.0 * c.M * c.N * c.K for c in host)
     weight_bytes = reps * R * sum(c.N * c.K / 4 for c in host)
     avg_launch_s = gemm_ms / 1e3 / launches
@@ -435,7 +448,7 @@ def run_ours(args):
     # ------------------------------------------------------------------ end to end through the public API
     pinned_x = [c.X.pin_memory() for c in host]
     pinned_u = [None if c.up is None else c.up.pin_memory() for c in host]
-    pinned_o = [torch.empty((c.M, c.N), dtype=torch.float32).pin_memory() for c in host]
+    pinned_o = [torch.empty((c.M, c.N), dtype=out_dtype).pin_memory() for c in host]
     e2e_steps = max(3, min(args.steps, 200))
     with torch.cuda.stream(stream):
         for _ in range(2):
@@ -462,7 +475,7 @@ def run_ours(args):
     e2e_ms = x0.elapsed_time(x1)
     e2e_max, e2e_tokens = aggregate(e2e_ms, e2e_steps * sum(c.M for c in host), world, dev)
     h2d = sum(in_bytes(c) for c in host)
-    d2h = sum(4 * c.M * c.N for c in host)
+    d2h = sum(out_bytes * c.M * c.N for c in host)
 
     result = None
     if rank == 0:
@@ -475,7 +488,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} copies ({R * step_bytes / 2**20:.0f} MiB > 4x L2)"
                        if R > 1 else "per-step working set larger than 4x L2",
-                       "cuda_graphs": True, "pdl": True},
+                       "cuda_graphs": True, "pdl": True, "out_dtype": args.out_dtype},
             "roofline": roof,
             "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
             "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
@@ -496,7 +509,7 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            v, desc, n, per_step = time_oracle(cases, budget_s=args.cpu_budget)
+            v, desc, n, per_step = time_oracle(cases, budget_s=args.cpu_budget, bf16_out=bf16_out)
             result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                       "sample": desc}
         print(json.dumps(result), flush=True)
@@ -729,15 +742,16 @@ def run_reference(args):
     cases = workload_cases(args.workload)
     budget = max(10.0, min(150.0, 6.0 * (args.steps + args.warmup)))
     # warm-up steps are untimed samples too; time exactly --steps steps
+    bf16_out = args.out_dtype == "bf16"
     if args.warmup:
-        time_oracle(cases, budget_s=budget, steps=1)
-    v, desc, n, per_step = time_oracle(cases, budget_s=budget, steps=args.steps)
+        time_oracle(cases, budget_s=budget, steps=1, bf16_out=bf16_out)
+    v, desc, n, per_step = time_oracle(cases, budget_s=budget, steps=args.steps, bf16_out=bf16_out)
     tokens = sum(c[1] for c in cases)
     result = {
         "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": workload_text(args.workload), "name": args.workload},
+        "config": {"workload": workload_text(args.workload), "name": args.workload, "out_dtype": args.out_dtype},
         "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": f"{tokens} tokens per step",
@@ -755,6 +769,8 @@ def main():
                     help="decode (default) | prefill | wdown | wdown_swiglu | msweep_M<M> | kvcache")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32",
+                    help="output storage of the forward workloads: fp32, or bf16 rounded to nearest even")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 4
+#define BITNET_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -167,6 +167,33 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype
                                           bitnet_act_mode_t mode, const uint8_t *packed,
                                           const float *alpha, int64_t N, float *out,
                                           void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * bf16-output variants.  The pages' epilogue (bitnet_v2_engine.py page, Eq. 5/6
+ * dequantisation; BitLinear_b158.forward's rescale) fixes the value, not the
+ * storage type; a bf16 output is this library's storage option.  The same
+ * computation as bitnet_ternary_gemm and
+ * bitnet_hbitlinear_forward, with the output written as
+ *   out_dt == BITNET_F32:   out[m][n] fp32, exactly as the calls above;
+ *   out_dt == BITNET_BF16:  out[m][n] = the fp32 value above rounded once to bf16,
+ *                           to nearest with ties to even (2 bytes per element),
+ * which halves the output stream.  out is [M][N] of out_dt, device, 16-byte
+ * aligned; any other out_dt is BITNET_ERR_INVALID_ARG.  The bf16 forward never
+ * splits K (its output cannot hold the int32 partial sums), so its plan can differ
+ * from bitnet_forward_gemm_plan's for few-tile, long-K shapes; the workspace is
+ * the same size.
+ * ------------------------------------------------------------------------ */
+BITNET_API bitnet_status_t bitnet_ternary_gemm_ex(const int8_t *codes, const float *scale_x,
+                                                  bitnet_act_mode_t mode, const uint8_t *packed,
+                                                  const float *alpha, int64_t M, int64_t N, int64_t K,
+                                                  void *out, bitnet_dtype_t out_dt, int32_t *acc_out,
+                                                  void *stream);
+BITNET_API bitnet_status_t bitnet_hbitlinear_forward_ex(const void *X, bitnet_dtype_t xdt, int64_t M,
+                                                        int64_t K, const float *gain, float eps, int fwht,
+                                                        bitnet_act_mode_t mode, const uint8_t *packed,
+                                                        const float *alpha, int64_t N, void *out,
+                                                        bitnet_dtype_t out_dt, void *ws, size_t ws_bytes,
+                                                        void *stream);
 
 /* --------------------------------------------------------------------------
  * SwiGLU-fused variants for the down projection of a BitNet v2 FFN.

@@ -36,7 +36,7 @@
  *   - The dequant epilogue is out = (float)acc * ((alpha * scale_x) / Q).
  *   - silu(g) = g / (1 + e^-g) in fp32 (the page calls F.silu = g * sigmoid(g)).
  *   - A bf16 output is the fp32 output rounded once to bf16, to nearest, ties to
- *     even (the pages name a bf16 output only as a storage option).
+ *     even (the pages fix the epilogue's value, not its storage type).
  */
 #include <math.h>
 #include <stdint.h>
@@ -372,7 +372,7 @@ int oracle_dequant(const int32_t *acc, const float *scale_x, float alpha, int mo
 }
 
 /* ---------------------------------------------------------------------------
- * bf16 output (NEXT row f4).  bf16 keeps the sign, the 8 exponent bits and the top
+ * bf16 output (NEXT row f4: a storage option for the epilogue's fp32 value).  bf16 keeps the sign, the 8 exponent bits and the top
  * 7 fraction bits of an fp32 value.  A finite x lies between two adjacent bf16
  * values: lo, x with its low 16 bits cleared (toward zero), and hi, the next one
  * away from zero.  The result is the nearer of the two; at the exact midpoint,

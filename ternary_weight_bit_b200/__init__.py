@@ -269,6 +269,60 @@ def bitnet_hbitlinear_forward_noalloc(X: torch.Tensor, packed: torch.Tensor, alp
     return out
 
 
+_OUT_DT = {torch.float32: 0, torch.bfloat16: 1}  # bitnet_dtype_t
+
+
+def _out_dt(dtype) -> int:
+    if dtype not in _OUT_DT:
+        raise ValueError(f"output dtype must be torch.float32 or torch.bfloat16, got {dtype}")
+    return _OUT_DT[dtype]
+
+
+def bitnet_ternary_gemm_ex(codes: torch.Tensor, scale_x: torch.Tensor, mode, packed: torch.Tensor,
+                           alpha: torch.Tensor, N: int, out_dtype=torch.bfloat16, out=None, acc_out=None,
+                           stream=None):
+    """bitnet_ternary_gemm with the output stored as out_dtype (fp32, or bf16 rounded to nearest even)."""
+    L = _native.load()
+    _need(codes, "codes", torch.int8)
+    M, K = codes.shape
+    _need(scale_x, "scale_x", torch.float32, (M,))
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(alpha, "alpha", torch.float32)
+    dt = _out_dt(out_dtype)
+    out = torch.empty((M, N), dtype=out_dtype, device=codes.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    if acc_out is not None:
+        _need(acc_out, "acc_out", torch.int32, (M, N))
+    _native.check("bitnet_ternary_gemm_ex",
+                  L.bitnet_ternary_gemm_ex(_ptr(codes), _ptr(scale_x), mode_id(mode), _ptr(packed), _ptr(alpha), M,
+                                           N, K, _ptr(out), dt, _ptr(acc_out), _stream(stream)))
+    return out
+
+
+def bitnet_hbitlinear_forward_ex(X: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, N: int, gain=None,
+                                 eps: float = 1e-5, fwht: bool = True, mode="int8", out_dtype=torch.bfloat16,
+                                 out=None, ws=None, stream=None):
+    """bitnet_hbitlinear_forward with the output stored as out_dtype (fp32, or bf16 rounded to nearest even)."""
+    L = _native.load()
+    _need(X, "X")
+    M, K = X.shape
+    _need(packed, "packed", torch.uint8, (N, K // 4))
+    _need(alpha, "alpha", torch.float32)
+    if gain is not None:
+        _need(gain, "gain", torch.float32, (K,))
+    dt = _out_dt(out_dtype)
+    out = torch.empty((M, N), dtype=out_dtype, device=X.device) if out is None else out
+    _need(out, "out", out_dtype, (M, N))
+    nbytes = L.bitnet_forward_workspace_bytes(M, K)
+    ws = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=X.device) if ws is None else ws
+    _need(ws, "ws", torch.uint8)
+    _native.check("bitnet_hbitlinear_forward_ex",
+                  L.bitnet_hbitlinear_forward_ex(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)),
+                                                 mode_id(mode), _ptr(packed), _ptr(alpha), N, _ptr(out), dt,
+                                                 _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
 def bitnet_get_last_device_status(stream=None) -> int:
     """Synchronise the stream, return and clear the kernels' timeout status word."""
     return _native.load().bitnet_get_last_device_status(_stream(stream))

@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_hbitlinear_forward_noalloc": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P]),
         "bitnet_act_quant_swiglu": (I, [P, P, I, I64, I64, P, F, I, I, P, P, P]),
         "bitnet_kv_quant": (I, [P, I, I64, I64, I64, I, F, P, P, P, P]),
+        "bitnet_ternary_gemm_ex": (I, [P, P, I, P, P, I64, I64, I64, P, I, P, P]),
+        "bitnet_hbitlinear_forward_ex": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, I, P, SZ, P]),
         "bitnet_hbitlinear_forward_swiglu": (I, [P, P, I, I64, I64, P, F, I, I, P, P, I64, P, P, SZ, P]),
         "bitnet_status_string": (ctypes.c_char_p, [I]),
         "bitnet_get_last_device_status": (I, [P]),

@@ -63,16 +63,17 @@ bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_x,
+bool make_tmap_out_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t cols, uint64_t rows, uint32_t box_x,
                       uint32_t box_y) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint64_t strides[1] = {cols * (bf16 ? 2 : 4)};
     const cuuint32_t box[2] = {box_x, box_y};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -113,7 +114,7 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, int *status) {
 }
 
 bitnet_status_t validate_gemm(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                              const float *alpha, int64_t M, int64_t N, int64_t K, const float *out,
+                              const float *alpha, int64_t M, int64_t N, int64_t K, const void *out,
                               const int32_t *acc_out) {
     if (mode != BITNET_ACT_INT8_ABSMAX && mode != BITNET_ACT_INT4_ABSMEAN) return BITNET_ERR_INVALID_ARG;
     if (M < 0 || N < 1 || M > kMaxRows || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
@@ -144,11 +145,13 @@ bitnet_status_t validate_act(const void *X, int xdt, int64_t M, int64_t K, const
 }
 
 cudaError_t run_gemm(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                     const float *alpha, int64_t M, int64_t N, int64_t K, float *out, int32_t *acc_out, bool pdl,
-                     cudaStream_t s) {
+                     const float *alpha, int64_t M, int64_t N, int64_t K, void *out, bool out_bf16,
+                     int32_t *acc_out, bool pdl, cudaStream_t s) {
     if (M <= kGemvMaxM)
-        return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s);
-    return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s);
+        return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s,
+                           out_bf16);
+    return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s,
+                          GemmPlan{0, 1}, nullptr, out_bf16);
 }
 
 }  // namespace
@@ -158,12 +161,13 @@ cudaError_t run_gemm(const int8_t *codes, const float *scale_x, int mode, const 
 // splits K: act_quant then also zeroes `out` and the tile counters for it.
 cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
                             int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
-                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
-                            const void *up) {
+                            int64_t N, void *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
+                            const void *up, bool out_bf16) {
     GemmPlan plan{0, 1};
     ZeroFill zf;
     if (M > kGemvMaxM) {
-        plan = gemm_plan((int)M, (int)N, (int)K, sm_count(), kSplitCounters);
+        // a bf16 output cannot hold the int32 sums of a split GEMM: never split it
+        plan = gemm_plan((int)M, (int)N, (int)K, sm_count(), out_bf16 ? 0 : kSplitCounters);
         if (plan.splits > 1) {
             zf.rows = reinterpret_cast<uint32_t *>(out);
             zf.row_words = (int)N;
@@ -176,9 +180,10 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
                        : launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s, zf);
     if (e != cudaSuccess) return e;
     if (M <= kGemvMaxM)
-        return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s);
+        return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s,
+                           out_bf16);
     return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s, plan,
-                          tile_cnt);
+                          tile_cnt, out_bf16);
 }
 
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s) {
@@ -239,8 +244,18 @@ bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x, b
                                     float *out, int32_t *acc_out, void *stream) {
     bitnet_status_t st = validate_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out);
     if (st != BITNET_OK || M == 0) return st;
-    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, true,
+    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, false, acc_out, true,
                               static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status_t bitnet_ternary_gemm_ex(const int8_t *codes, const float *scale_x, bitnet_act_mode_t mode,
+                                       const uint8_t *packed, const float *alpha, int64_t M, int64_t N, int64_t K,
+                                       void *out, bitnet_dtype_t out_dt, int32_t *acc_out, void *stream) {
+    if (out_dt != BITNET_F32 && out_dt != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+    bitnet_status_t st = validate_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out);
+    if (st != BITNET_OK || M == 0) return st;
+    return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, out_dt == BITNET_BF16, acc_out,
+                              true, static_cast<cudaStream_t>(stream)));
 }
 
 size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K) {
@@ -253,7 +268,8 @@ size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K) {
 namespace {
 bitnet_status_t forward_ws(const void *X, const void *up, bitnet_dtype_t xdt, int64_t M, int64_t K,
                            const float *gain, float eps, int fwht, bitnet_act_mode_t mode, const uint8_t *packed,
-                           const float *alpha, int64_t N, float *out, void *ws, size_t ws_bytes, void *stream) {
+                           const float *alpha, int64_t N, void *out, bool out_bf16, void *ws, size_t ws_bytes,
+                           void *stream) {
     if (N < 1 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
     bitnet_status_t st = validate_act(X, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
     if (st != BITNET_OK || M == 0) return st;
@@ -265,7 +281,7 @@ bitnet_status_t forward_ws(const void *X, const void *up, bitnet_dtype_t xdt, in
     float *scale_x = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)M * (size_t)K));
     int *tile_cnt = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(scale_x) + align256((size_t)M * sizeof(float)));
     return from_cuda(forward_kernels(X, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, codes, scale_x,
-                                     tile_cnt, static_cast<cudaStream_t>(stream), up));
+                                     tile_cnt, static_cast<cudaStream_t>(stream), up, out_bf16));
 }
 }  // namespace
 
@@ -273,7 +289,17 @@ bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int
                                           const float *gain, float eps, int fwht, bitnet_act_mode_t mode,
                                           const uint8_t *packed, const float *alpha, int64_t N, float *out,
                                           void *ws, size_t ws_bytes, void *stream) {
-    return forward_ws(X, nullptr, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, ws, ws_bytes, stream);
+    return forward_ws(X, nullptr, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, false, ws, ws_bytes,
+                      stream);
+}
+
+bitnet_status_t bitnet_hbitlinear_forward_ex(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                             const float *gain, float eps, int fwht, bitnet_act_mode_t mode,
+                                             const uint8_t *packed, const float *alpha, int64_t N, void *out,
+                                             bitnet_dtype_t out_dt, void *ws, size_t ws_bytes, void *stream) {
+    if (out_dt != BITNET_F32 && out_dt != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+    return forward_ws(X, nullptr, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, out_dt == BITNET_BF16,
+                      ws, ws_bytes, stream);
 }
 
 bitnet_status_t bitnet_act_quant_swiglu(const void *gate, const void *up, bitnet_dtype_t xdt, int64_t M, int64_t K,
@@ -295,7 +321,7 @@ bitnet_status_t bitnet_hbitlinear_forward_swiglu(const void *gate, const void *u
         const bitnet_status_t st = validate_act(gate, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
         return st != BITNET_OK ? st : BITNET_ERR_INVALID_ARG;
     }
-    return forward_ws(gate, up, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, ws, ws_bytes, stream);
+    return forward_ws(gate, up, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, false, ws, ws_bytes, stream);
 }
 
 int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {

@@ -30,8 +30,8 @@
 //                likewise warp-uniform with elected issue
 //   UW sets of 4 unpack warps; set u takes the stages it with it % UW == u.  Warp w
 //                owns TMEM lanes 32 (w % 4) .. +31 (= weight rows) of its slot.
-//   4 epilogue warps: tcgen05.ld, out[m][n] = acc * f[m]; the fp32 tile goes out
-//                through shared memory with one TMA bulk tensor store per 32 tokens.
+//   4 epilogue warps: tcgen05.ld, out[m][n] = acc * f[m]; the fp32 (or bf16) tile goes
+//                out through shared memory with one TMA bulk tensor store per 32 tokens.
 // All waits are bounded; a timeout is recorded in the device status word.
 #include <string.h>
 
@@ -54,7 +54,7 @@ struct TcCfg {
     static constexpr int P_BYTES = BW * BK / 4;  // packed weight tile (4 KB)
     static constexpr int B_OFF = 0;
     static constexpr int P_OFF = ST * B_BYTES;
-    static constexpr int O_OFF = P_OFF + ST * P_BYTES;             // 2 x [32 tokens][128 rows] fp32
+    static constexpr int O_OFF = P_OFF + ST * P_BYTES;             // 2 x [32 tokens][128 rows] fp32 or bf16
     static constexpr int F_OFF = O_OFF + 2 * OUT_TOKENS * BW * 4;  // per-token dequant factors, DB rows
     static constexpr int BAR_OFF = F_OFF + DB * BT * 4;
     static constexpr int NUM_BARS = 2 * ST + 2 * AS + 2 * DB;
@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_out, int tma_out, const uint8_t *__restrict__ packed,
                const float *__restrict__ scale_x,
-               const float *__restrict__ alpha, int mode, int M, int N, int K, float *__restrict__ out,
-               int32_t *__restrict__ acc_out, int splits, int *__restrict__ tile_cnt, int *status) {
+               const float *__restrict__ alpha, int mode, int M, int N, int K, void *__restrict__ out_v,
+               int out_bf16, int32_t *__restrict__ acc_out, int splits, int *__restrict__ tile_cnt, int *status) {
     constexpr int BT = C::BT, ST = C::ST, AS = C::AS, DB = C::DB, UW = C::UW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,6 +322,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
         const int et = threadIdx.x - (64 + 128 * UW);  // 0..127
         float *obuf = reinterpret_cast<float *>(smem + C::O_OFF);
         const uint32_t sO0 = smem_u32(obuf);
+        float *out = reinterpret_cast<float *>(out_v);                   // fp32 output (and split-K image)
+        __nv_bfloat16 *outh = reinterpret_cast<__nv_bfloat16 *>(out_v);  // bf16 output (never split)
+        const int obytes = out_bf16 ? 2 : 4;
         if (et == 0 && tma_out) tma_prefetch_desc(&tm_out);
         pdl_wait_prerequisites();
         const float a_scale = *alpha;
@@ -401,14 +404,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
                     const int buf = ck & 1;
                     if (et == 0 && ck >= 2) bulk_wait_group_read<1>();  // the store that read buf is done
                     asm volatile("bar.sync 1, 128;" ::: "memory");
-                    float *sb = obuf + buf * (OUT_TOKENS * BW);
+                    if (out_bf16) {
+                        __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(obuf) + buf * (OUT_TOKENS * BW);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        sb[j * BW + r] = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                        for (int j = 0; j < 32; ++j)
+                            sb[j * BW + r] = __float2bfloat16_rn(__fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]));
+                    } else {
+                        float *sb = obuf + buf * (OUT_TOKENS * BW);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            sb[j * BW + r] = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                    }
                     fence_proxy_async_smem();
                     asm volatile("bar.sync 1, 128;" ::: "memory");
                     if (et == 0) {
-                        tma_store_2d(&tm_out, sO0 + (uint32_t)(buf * OUT_TOKENS * BW * 4), n0, m0 + 32 * c);
+                        tma_store_2d(&tm_out, sO0 + (uint32_t)(buf * OUT_TOKENS * BW * obytes), n0, m0 + 32 * c);
                         bulk_commit_group();
                     }
                     ++ck;
@@ -416,7 +426,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int m = m0 + 32 * c + j;
-                        if (m < M) out[(int64_t)m * N + n] = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                        if (m >= M) continue;
+                        const float y = __fmul_rn((float)(int)v[j], fac[b * BT + 32 * c + j]);
+                        if (out_bf16) outh[(int64_t)m * N + n] = __float2bfloat16_rn(y);
+                        else out[(int64_t)m * N + n] = y;
                     }
                 }
                 if (acc_out && n < N) {
@@ -445,8 +458,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
 
 template <class C>
 cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                       const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, int splits,
-                       int *tile_cnt, bool pdl, cudaStream_t s) {
+                       const float *alpha, int M, int N, int K, void *out, bool out_bf16, int32_t *acc_out,
+                       int splits, int *tile_cnt, bool pdl, cudaStream_t s) {
     CUtensorMap ta, tw, to;
     if (!make_tmap_u8_2d(&ta, codes, (uint64_t)K, (uint64_t)M, BK, C::BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -454,9 +467,11 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
         return cudaErrorInvalidValue;
     // The bulk-store epilogue needs a 16-byte row pitch and base, and a box that fits.
     memset(&to, 0, sizeof(to));
-    const bool store_ok = splits == 1 && N % 4 == 0 && M >= OUT_TOKENS && N >= BW &&
+    // (N elements of 4 or 2 bytes per row: N % 4 == 0 for fp32, N % 8 == 0 for bf16)
+    const bool store_ok = splits == 1 && N % (out_bf16 ? 8 : 4) == 0 && M >= OUT_TOKENS && N >= BW &&
                           (reinterpret_cast<uintptr_t>(out) & 15) == 0;
-    const int tma_out = store_ok && make_tmap_f32_2d(&to, out, (uint64_t)N, (uint64_t)M, BW, OUT_TOKENS) ? 1 : 0;
+    const int tma_out =
+        store_ok && make_tmap_out_2d(&to, out, out_bf16, (uint64_t)N, (uint64_t)M, BW, OUT_TOKENS) ? 1 : 0;
     auto kern = gemm_tc_kernel<C>;
     static bool done[kMaxDevices] = {};
     int dev = 0;
@@ -479,8 +494,8 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, packed, scale_x, alpha, mode, M, N, K, out, acc_out,
-                              splits, tile_cnt, device_status_ptr());
+    return cudaLaunchKernelEx(&cfg, kern, ta, tw, to, tma_out, packed, scale_x, alpha, mode, M, N, K, out,
+                              out_bf16 ? 1 : 0, acc_out, splits, tile_cnt, device_status_ptr());
 }
 
 }  // namespace
@@ -536,17 +551,18 @@ GemmPlan gemm_plan(int M, int N, int K, int sms, int max_split_tiles) {
 int gemm_pick_tile(int M, int N, int K, int sms) { return gemm_plan(M, N, K, sms, 0).token_tile; }
 
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                           const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
-                           cudaStream_t s, GemmPlan plan, int *tile_cnt) {
+                           const float *alpha, int M, int N, int K, void *out, int32_t *acc_out, bool pdl,
+                           cudaStream_t s, GemmPlan plan, int *tile_cnt, bool out_bf16) {
     if (plan.token_tile == 0) plan = gemm_plan(M, N, K, sm_count(), 0);
     const int sp = plan.splits;
-    if (sp < 1 || (sp > 1 && (!tile_cnt || (K / BK) % sp != 0))) return cudaErrorInvalidValue;
+    // a split GEMM accumulates int32 in the output itself, which a bf16 output cannot hold
+    if (sp < 1 || (sp > 1 && (!tile_cnt || (K / BK) % sp != 0 || out_bf16))) return cudaErrorInvalidValue;
     switch (plan.token_tile) {
-    case 256: return launch_cfg<Cfg256>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
-    case 224: return launch_cfg<Cfg224>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
-    case 192: return launch_cfg<Cfg192>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
-    case 128: return launch_cfg<Cfg128>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
-    case 64: return launch_cfg<Cfg64>(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out, sp, tile_cnt, pdl, s);
+    case 256: return launch_cfg<Cfg256>(codes, scale_x, mode, packed, alpha, M, N, K, out, out_bf16, acc_out, sp, tile_cnt, pdl, s);
+    case 224: return launch_cfg<Cfg224>(codes, scale_x, mode, packed, alpha, M, N, K, out, out_bf16, acc_out, sp, tile_cnt, pdl, s);
+    case 192: return launch_cfg<Cfg192>(codes, scale_x, mode, packed, alpha, M, N, K, out, out_bf16, acc_out, sp, tile_cnt, pdl, s);
+    case 128: return launch_cfg<Cfg128>(codes, scale_x, mode, packed, alpha, M, N, K, out, out_bf16, acc_out, sp, tile_cnt, pdl, s);
+    case 64: return launch_cfg<Cfg64>(codes, scale_x, mode, packed, alpha, M, N, K, out, out_bf16, acc_out, sp, tile_cnt, pdl, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -52,8 +52,8 @@ struct Chunk {
 template <int WK, int NT, int PF>  // PF: chunks of loads in flight per warp
 __global__ void __launch_bounds__(32 * WK)
 gemv_kernel(const uint8_t *__restrict__ packed, const int8_t *__restrict__ codes, const float *__restrict__ scale_x,
-            const float *__restrict__ alpha, int mode, int M, int N, int K, float *__restrict__ out,
-            int32_t *__restrict__ acc_out) {
+            const float *__restrict__ alpha, int mode, int M, int N, int K, void *__restrict__ out,
+            int out_bf16, int32_t *__restrict__ acc_out) {
     constexpr int TOK = 8 * NT;
     __shared__ int32_t red[WK][ROWS * TOK];
     __shared__ float fac[TOK];
@@ -163,7 +163,11 @@ gemv_kernel(const uint8_t *__restrict__ packed, const int8_t *__restrict__ codes
             int32_t sum = 0;
 #pragma unroll
             for (int w = 0; w < WK; ++w) sum += red[w][r * TOK + tok];
-            out[(int64_t)tok * N + n] = __fmul_rn((float)sum, fac[tok]);
+            const float y = __fmul_rn((float)sum, fac[tok]);
+            if (out_bf16)  // the fp32 value rounded once, to nearest even
+                reinterpret_cast<__nv_bfloat16 *>(out)[(int64_t)tok * N + n] = __float2bfloat16_rn(y);
+            else
+                reinterpret_cast<float *>(out)[(int64_t)tok * N + n] = y;
             if (acc_out) acc_out[(int64_t)tok * N + n] = sum;
         }
     }
@@ -171,7 +175,7 @@ gemv_kernel(const uint8_t *__restrict__ packed, const int8_t *__restrict__ codes
 
 template <int WK, int NT, int PF>
 cudaError_t launch_cfg(const uint8_t *packed, const int8_t *codes, const float *scale_x, int mode, const float *alpha,
-                       int M, int N, int K, float *out, int32_t *acc_out, bool pdl, cudaStream_t s) {
+                       int M, int N, int K, void *out, bool out_bf16, int32_t *acc_out, bool pdl, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((N + ROWS - 1) / ROWS));
     cfg.blockDim = dim3(32 * WK);
@@ -182,23 +186,24 @@ cudaError_t launch_cfg(const uint8_t *packed, const int8_t *codes, const float *
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<WK, NT, PF>, packed, codes, scale_x, alpha, mode, M, N, K, out, acc_out);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<WK, NT, PF>, packed, codes, scale_x, alpha, mode, M, N, K, out,
+                              out_bf16 ? 1 : 0, acc_out);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                        const float *alpha, int M, int N, int K, float *out, int32_t *acc_out, bool pdl,
-                        cudaStream_t s) {
+                        const float *alpha, int M, int N, int K, void *out, int32_t *acc_out, bool pdl,
+                        cudaStream_t s, bool out_bf16) {
     const int nch = (K + 255) / 256;
     // 4 warps per 16-row block for short K, 8 when each warp would otherwise own many chunks
     const int wk = nch <= 16 ? 4 : 8;
     if (M <= 8) {
-        if (wk == 4) return launch_cfg<4, 1, 3>(packed, codes, scale_x, mode, alpha, M, N, K, out, acc_out, pdl, s);
-        return launch_cfg<8, 1, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, acc_out, pdl, s);
+        if (wk == 4) return launch_cfg<4, 1, 3>(packed, codes, scale_x, mode, alpha, M, N, K, out, out_bf16, acc_out, pdl, s);
+        return launch_cfg<8, 1, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, out_bf16, acc_out, pdl, s);
     }
-    if (wk == 4) return launch_cfg<4, 2, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, acc_out, pdl, s);
-    return launch_cfg<8, 2, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, acc_out, pdl, s);
+    if (wk == 4) return launch_cfg<4, 2, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, out_bf16, acc_out, pdl, s);
+    return launch_cfg<8, 2, 2>(packed, codes, scale_x, mode, alpha, M, N, K, out, out_bf16, acc_out, pdl, s);
 }
 
 }  // namespace bitnet

@@ -19,9 +19,9 @@ constexpr int kGemvMaxM = 16;
 bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uint64_t rows,
                      uint32_t box_x, uint32_t box_y, CUtensorMapSwizzle swizzle);
 
-// 2D fp32 tensor map (no swizzle) over a row-major [rows][cols] array; cols * 4 and
-// the base must be 16-byte aligned.
-bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_x,
+// 2D fp32 or bf16 tensor map (no swizzle) over a row-major [rows][cols] array; the row
+// pitch and the base must be 16-byte aligned.
+bool make_tmap_out_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t cols, uint64_t rows, uint32_t box_x,
                       uint32_t box_y);
 
 // Per-device address of the library's device status word.
@@ -51,24 +51,27 @@ cudaError_t launch_pack(const float *W, int64_t N, int64_t K, float eps, uint8_t
                         void *ws, cudaStream_t s);
 
 // Decode path (M <= 16): weight-streaming kernel, 2-bit weights unpacked in
-// registers, int8 mma.sync, split-K over the warps of one CTA.
+// registers, int8 mma.sync, split-K over the warps of one CTA.  `out` is fp32, or
+// bf16 when out_bf16 (the fp32 value rounded to nearest even).
 cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                        const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
-                        bool pdl, cudaStream_t s);
+                        const float *alpha, int M, int N, int K, void *out, int32_t *acc_out,
+                        bool pdl, cudaStream_t s, bool out_bf16 = false);
 
 // Prefill path: tcgen05 int8 tensor-core GEMM with TMEM accumulators.
 // A plan is a token-tile size (256/224/192/128/64) and a k-split count (1, 2, 4, 8).
 // With splits > 1, `out` must be zero on entry (the kernel adds int32 partial sums
 // into it before dequantising in place) and tile_cnt must point at
-// kSplitCounters zeroed ints (the kernel leaves them zero again).
+// kSplitCounters zeroed ints (the kernel leaves them zero again).  A bf16 output
+// (out_bf16) is never split.
 struct GemmPlan {
     int token_tile;  // 0: choose automatically (no split)
     int splits;
 };
 constexpr int kSplitCounters = 1024;
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
-                           const float *alpha, int M, int N, int K, float *out, int32_t *acc_out,
-                           bool pdl, cudaStream_t s, GemmPlan plan = GemmPlan{0, 1}, int *tile_cnt = nullptr);
+                           const float *alpha, int M, int N, int K, void *out, int32_t *acc_out,
+                           bool pdl, cudaStream_t s, GemmPlan plan = GemmPlan{0, 1}, int *tile_cnt = nullptr,
+                           bool out_bf16 = false);
 
 // The plan launch_gemm_tc uses for this shape on `sms` SMs; splits > 1 only when the
 // output has at most max_split_tiles tiles (0: never split).  Honors a forced tile.
@@ -81,11 +84,12 @@ bool gemm_force_tile(int bt);
 
 // The forward's kernels (act_quant, then GEMV or GEMM), arguments validated;
 // tile_cnt points at kSplitCounters ints of workspace for a split-K GEMM.  With
-// `up` given, X is the SwiGLU gate and the input is silu(X) * up.
+// `up` given, X is the SwiGLU gate and the input is silu(X) * up.  `out` is fp32,
+// or bf16 when out_bf16.
 cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
                             int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
-                            int64_t N, float *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
-                            const void *up = nullptr);
+                            int64_t N, void *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
+                            const void *up = nullptr, bool out_bf16 = false);
 
 // Low-bit KV cache: kv [BH][S][D] (fp32 or bf16), D % 4 == 0, D <= 1024; bits 3, 4 or 8
 // for tokens s >= 1 (token 0 is always int8).  deq may be null.

@@ -93,3 +93,25 @@ def check_out_end_to_end(gpu_out, ora_out, gpu_codes, ora_codes, ora_scale, alph
     assert len(bad) == 0, (f"{label}: token {bad[0]} err {err[bad[0]]:.3g} > bound {bound[bad[0]]:.3g} "
                            f"(flips {flips[bad[0]]})")
     assert float((err / np.maximum(ref, 1e-30)).max()) <= OUT_RTOL + float((flips * step / np.maximum(ref, 1e-30)).max())
+
+
+def bf16_bits(t):
+    """uint16 bit patterns of a bf16 torch tensor (on any device)."""
+    return t.detach().contiguous().view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_values(bits):
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32)
+
+
+def check_out_end_to_end_bf16(gpu_bits, ora_out, gpu_codes, ora_codes, ora_scale, alpha, mode, label=""):
+    """The fp32 bound of check_out_end_to_end plus the bf16 rounding of each element
+    (at most half a bf16 step, 2^-9 of the value, taken as 2^-8 of the oracle's)."""
+    g = bf16_values(gpu_bits).astype(np.float64)
+    flips = (gpu_codes != ora_codes).sum(axis=1)
+    step = np.float64(alpha) * ora_scale.astype(np.float64) / float(q_of(mode))
+    ref = np.abs(ora_out).max(axis=1)
+    bound = (OUT_RTOL * ref + flips * step * 1.001)[:, None] + 2.0 ** -8 * np.abs(ora_out) + 1e-30
+    bad = np.argwhere(np.abs(g - ora_out) > bound)
+    assert len(bad) == 0, f"{label}: element {tuple(bad[0])} outside the bf16 end-to-end bound"
+

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 4
+    assert L.bitnet_abi_version() == 5
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
@@ -64,6 +64,20 @@ def test_kv_quant_validation(L):
     assert L.bitnet_kv_quant(None, 0, 0, 3, 128, 3, 1e-5, None, None, None, s) == ok   # empty: nothing to do
     assert L.bitnet_kv_quant(None, 0, 2, 3, 128, 3, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG
     assert L.bitnet_kv_quant(P(4100), 0, 2, 3, 128, 3, 1e-5, FAKE, FAKE, None, s) == _native.ERR_INVALID_ARG
+
+
+def test_out_dtype_validation(L):
+    s = P(0)
+    # an output dtype other than fp32 / bf16 is refused before anything else is looked at
+    assert L.bitnet_ternary_gemm_ex(FAKE, FAKE, 0, FAKE, FAKE, 4, 256, 256, FAKE, 2, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_hbitlinear_forward_ex(FAKE, 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, 256, FAKE, 7, FAKE, 1 << 20,
+                                          s) == _native.ERR_INVALID_ARG
+    # the shape checks still apply with a valid output dtype
+    assert L.bitnet_ternary_gemm_ex(FAKE, FAKE, 0, FAKE, FAKE, 4, 256, 100, FAKE, 1, None, s) == \
+        _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_hbitlinear_forward_ex(FAKE, 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, 256, P(4100), 1, FAKE,
+                                          1 << 20, s) == _native.ERR_INVALID_ARG  # misaligned out
+    assert L.bitnet_ternary_gemm_ex(None, None, 0, None, None, 0, 256, 256, None, 1, None, s) == _native.OK  # M = 0
 
 
 def test_workspace_sizes(L):

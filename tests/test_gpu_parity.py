@@ -201,6 +201,89 @@ def test_gemm_extreme_codes():
         np.testing.assert_array_equal(host(acc), ref.gemm_packed(q, packed, N))
 
 
+# ----------------------------------------------------------------------------- bf16 output
+BF16_GEMM_SHAPES = [
+    (1, 64, 128), (5, 700, 2560), (8, 6912, 2560), (16, 512, 1024),           # decode kernel
+    (17, 256, 128), (130, 300, 384), (300, 1000, 2048), (2048, 2560, 256),    # tcgen05, bulk-store epilogue
+    (77, 130, 384), (64, 1990, 256), (1051, 4100, 256),                      # N % 8 != 0: direct stores
+]
+
+
+@pytest.mark.parametrize("M,N,K", BF16_GEMM_SHAPES)
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_gemm_bf16_output_exact(M, N, K, mode):
+    # the bf16 output is the oracle's fp32 epilogue value rounded once, bit for bit
+    q, packed, scale, alpha = _gemm_case(M, N, K, mode, seed=M * 31 + N + K)
+    acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    out = tb.bitnet_ternary_gemm_ex(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, out_dtype=torch.bfloat16,
+                                    acc_out=acc)
+    assert out.dtype == torch.bfloat16
+    acc_ref = ref.gemm_packed(q, packed, N)
+    np.testing.assert_array_equal(host(acc), acc_ref)
+    want = ref.round_bf16(ref.dequant(acc_ref, scale, alpha[0], MODES[mode]))
+    np.testing.assert_array_equal(parity.bf16_bits(out), want, err_msg=f"{M}x{N}x{K} {mode}")
+    # the fp32 choice of the same entry point is the plain GEMM
+    out32 = tb.bitnet_ternary_gemm_ex(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, out_dtype=torch.float32)
+    np.testing.assert_array_equal(host(out32), ref.dequant(acc_ref, scale, alpha[0], MODES[mode]))
+
+
+@pytest.mark.parametrize("tile", [256, 224, 192, 128, 64])
+def test_gemm_bf16_output_forced_tiles(tile):
+    try:
+        tb.bitnet_gemm_force_token_tile(tile)
+        for i, (M, N, K) in enumerate([(6 * tile + 45, 1032, 256), (40, 136, 128)]):
+            mode = ("int4", "int8")[i]
+            q, packed, scale, alpha = _gemm_case(M, N, K, mode, seed=tile + i)
+            out = tb.bitnet_ternary_gemm_ex(dev(q), dev(scale), mode, dev(packed), dev(alpha), N)
+            want = ref.round_bf16(ref.dequant(ref.gemm_packed(q, packed, N), scale, alpha[0], MODES[mode]))
+            np.testing.assert_array_equal(parity.bf16_bits(out), want, err_msg=f"tile {tile} {M}x{N}x{K}")
+    finally:
+        tb.bitnet_gemm_force_token_tile(0)
+
+
+def _forward_case_bf16(case, sample_rows=None):
+    Xd = case.X.to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(case.W.to(DEV), eps=case.eps)
+    out = tb.bitnet_hbitlinear_forward_ex(Xd, packed, alpha, case.N, eps=case.eps, fwht=case.fwht, mode=case.mode,
+                                          out_dtype=torch.bfloat16)
+    codes, gscale = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=case.fwht, mode=case.mode)
+    torch.cuda.synchronize()
+    rows = np.arange(case.M) if sample_rows is None else sample_rows
+    X32 = case.X.float().numpy()[rows]
+    p_ref, a_ref, _ = ref.pack_weights(case.W.numpy(), eps=case.eps)
+    np.testing.assert_array_equal(host(packed), p_ref)
+    mode = MODES[case.mode]
+    r = ref.hbitlinear_forward(X32, p_ref, a_ref, case.N, eps=case.eps, fwht_on=case.fwht, mode=mode)
+    sh = ref.shadow(X32, None, case.eps, case.fwht, mode)
+    gcodes = host(codes)[rows]
+    parity.check_codes(gcodes, r.codes, sh, case.name)
+    gs = host(gscale)[rows]
+    parity.check_scale_bound(gs, r.scale_x, case.K, mode, case.name)
+    gbits = parity.bf16_bits(out)[rows]
+    # same codes and scales -> the same fp32 value, rounded once to the same bf16
+    want = ref.round_bf16(ref.dequant(ref.gemm_packed(gcodes, p_ref, case.N), gs, a_ref, mode))
+    np.testing.assert_array_equal(gbits, want, err_msg=case.name)
+    parity.check_out_end_to_end_bf16(gbits, r.out, gcodes, r.codes, r.scale_x, a_ref, mode, case.name)
+
+
+@pytest.mark.parametrize("M,K,N,mode,fwht,xdt", [
+    (1, 2560, 6912, "int8", False, "f32"),    # decode kernel
+    (8, 6912, 2560, "int8", False, "f32"),
+    (100, 1024, 300, "int4", True, "f32"),    # tcgen05, N % 8 != 0
+    (257, 2048, 520, "int8", False, "bf16"),  # bulk-store epilogue
+    (64, 16384, 4096, "int4", True, "f32"),   # a shape the fp32 forward splits over K; bf16 never splits
+])
+def test_forward_bf16_output(M, K, N, mode, fwht, xdt):
+    case = synthetic.make_case("bf16out", M, K, N, x_kind="student_t3", outliers=max(1, K // 100),
+                               outlier_gain=50.0, x_dtype=xdt, fwht=fwht, mode=mode, seed=M + K + N)
+    _forward_case_bf16(case, None if M <= 300 else _sample(M, 24))
+
+
+def test_forward_bf16_output_prefill_sampled():
+    case = synthetic.prefill_int8(M=4096, K=4096, N=4096, fwht=True)
+    _forward_case_bf16(case, _sample(case.M, 16))
+
+
 # ----------------------------------------------------------------------------- whole forward
 def _forward_case(case, sample_rows=None):
     Xd = case.X.to(DEV)
