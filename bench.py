@@ -445,6 +445,39 @@ def run_ours(args):
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
                 "ops_per_launch": round(gemm_ops / launches)}
 
+    # ------------------------------------------------------------------ activation kernel alone
+    # (rows RMSNorm / FWHT / quantise): one graph over every case and rotation, into the
+    # codes and scales above; algorithmic bytes = X (and up) in, codes and scales out
+    def act_pass(r):
+        for c, (codes, scale), (X, p, a, out, ws, U) in zip(host, codes_scales, rot[r]):
+            if U is None:
+                tb.bitnet_act_quant(X, eps=c.eps, fwht=c.fwht, mode=c.mode, codes=codes, scale_x=scale)
+            else:
+                tb.bitnet_act_quant_swiglu(X, U, eps=c.eps, fwht=c.fwht, mode=c.mode, codes=codes, scale_x=scale)
+
+    ga = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ga, stream=stream):
+        for r in range(R):
+            act_pass(r)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ga.replay()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            ga.replay()
+    a1.record(stream)
+    a1.synchronize()
+    act_s = a0.elapsed_time(a1) / 1e3 / (reps * R * len(host))
+    act_bytes = sum(in_bytes(c) + c.M * c.K + 4 * c.M for c in host) / len(host)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    act = {"kernel": "act_quant (RMSNorm, FWHT when on, int8/int4 codes)", "bound": "hbm",
+           "avg_launch_us": round(act_s * 1e6, 3), "bytes_per_launch": round(act_bytes),
+           "achieved": round(act_bytes / act_s / 1e9, 1), "peak": hbm, "unit": "GB/s",
+           "frac": round(act_bytes / act_s / 1e9 / hbm, 4)}
+
     # ------------------------------------------------------------------ end to end through the public API
     pinned_x = [c.X.pin_memory() for c in host]
     pinned_u = [None if c.up is None else c.up.pin_memory() for c in host]
@@ -490,6 +523,7 @@ def run_ours(args):
                        if R > 1 else "per-step working set larger than 4x L2",
                        "cuda_graphs": True, "pdl": True, "out_dtype": args.out_dtype},
             "roofline": roof,
+            "act_quant": act,
             "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
             "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
             "e2e": {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",

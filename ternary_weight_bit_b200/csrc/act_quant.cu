@@ -63,20 +63,10 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 // ------------------------------------------------------------------ quantiser
-// Round-clip y*s to [lo, hi] with round-half-to-even, returned as the low byte of
-// the result: adding 1.5*2^23 rounds an fp32 in [-2^22, 2^22] to the nearest
-// integer (ties to even) and leaves that integer in the low mantissa bits.
-__device__ __forceinline__ uint32_t quant_byte(float y, float s, float lo, float hi) {
-    const float v = fminf(fmaxf(__fmul_rn(y, s), lo), hi);
-    return __float_as_uint(__fadd_rn(v, 12582912.0f)) & 0xFFu;
-}
-
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-    return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-}
-
-// As quant_byte, but returns the whole rounded word (code in the low byte) and
-// clips only when asked.
+// Round-clip y*s to [lo, hi] with round-half-to-even: adding 1.5*2^23 rounds an fp32
+// in [-2^22, 2^22] to the nearest integer (ties to even) and leaves that integer in
+// the low mantissa bits.  Returns the whole word (code in the low byte); clips only
+// when asked.
 __device__ __forceinline__ uint32_t quant_bits(float y, float s, float lo, float hi, bool clip) {
     float v = __fmul_rn(y, s);
     if (clip) v = fminf(fmaxf(v, lo), hi);
@@ -218,11 +208,11 @@ __device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
 // Zero the token's row of a following split-K GEMM's output (it adds int32 partial
 // sums there) and, in CTA 0, that GEMM's tile counters.  Runs after the dependency
 // wait: the buffers may still be read by earlier kernels until then.
-__device__ __forceinline__ void zero_fill(const ZeroFill &z) {
+__device__ __forceinline__ void zero_fill(const ZeroFill &z, int64_t token) {
     if (!z.rows) return;
-    uint32_t *row = z.rows + (int64_t)blockIdx.x * z.row_words;
+    uint32_t *row = z.rows + token * z.row_words;
     for (int i = threadIdx.x; i < z.row_words; i += blockDim.x) row[i] = 0u;
-    if (blockIdx.x == 0)
+    if (token == 0)
         for (int i = threadIdx.x; i < z.cnt_n; i += blockDim.x) z.cnt[i] = 0;
 }
 
@@ -240,7 +230,7 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
     // reads the codes, so the order of the data is kept.
     pdl_launch_dependents();
     pdl_wait_prerequisites();
-    zero_fill(zf);
+    zero_fill(zf, blockIdx.x);
 
     const int tid = threadIdx.x;
     const int64_t row = (int64_t)blockIdx.x * K;
@@ -345,68 +335,154 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
 }
 
 // ------------------------------------------------------------------ plain kernel (no FWHT)
-// Thread tid owns the float4 groups j = it*T + tid, it in [0, NV); K % 4 == 0.
-template <int T, int NV, class Src>
-__global__ void __launch_bounds__(T)
+// Per-token scalars of the plain kernel, computed once by warp 0 and shared.
+struct TokenScalars {
+    float rn, stat, s, lo, hi;
+};
+
+// Block reduction of (sum, max-or-sum) over a CTA of any whole number of warps.  Every
+// warp reduces its own values with shuffles; warp 0 combines the per-warp results and
+// runs finish(r) on its lane 0, which writes the token's scalars to *out; the CTA then
+// synchronises, so every thread may read *out.
+template <class F>
+__device__ __forceinline__ void block_reduce2(float ss, float st, bool mean, float2 *red, F finish) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float t = __shfl_xor_sync(0xffffffffu, st, o);
+        st = mean ? st + t : fmaxf(st, t);
+    }
+    const int W = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();  // red and the scalars may still be read from a previous reduction
+    if (lane == 0) red[warp] = make_float2(ss, st);
+    __syncthreads();
+    if (warp == 0) {
+        float2 r = lane < W ? red[lane] : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            r.x += __shfl_xor_sync(0xffffffffu, r.x, o);
+            const float t = __shfl_xor_sync(0xffffffffu, r.y, o);
+            r.y = mean ? r.y + t : fmaxf(r.y, t);
+        }
+        if (lane == 0) finish(r);
+    }
+    __syncthreads();
+}
+
+// One CTA of T threads (a multiple of 32, chosen per K and M) per token; thread tid
+// owns the 8-element chunks c = it*T + tid, it in [0, NV8); K % 8 == 0.  Without a
+// gain the statistics of y = x * r come from those of x in the same pass as sum(x^2):
+//   int8:  max_k |fl(x_k r)| = fl(r max_k |x_k|)   (rounding is monotone), exact;
+//   int4:  sum_k |fl(x_k r)| = fl(r sum_k |x_k|) up to one rounding per term,
+// so one block reduction serves both.  With a gain, y is formed first and reduced
+// again.  The scalar steps (IEEE divisions and square root) run once per token, in one
+// thread.  Per element the kernel then spends two multiplies, one add and a byte
+// permute on the code.
+template <int NV8, class Src>
+__global__ void __launch_bounds__(512)
 act_quant_plain_kernel(Src src, const float *__restrict__ gain, int K, float eps,
                        int mode, int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
-    __shared__ float red[32];
+    __shared__ float2 red[32];
+    __shared__ TokenScalars ts;
     pdl_launch_dependents();  // as in the FWHT kernel: the GEMM may launch, X is waited for
     pdl_wait_prerequisites();
-    zero_fill(zf);
-    const int tid = threadIdx.x;
+    zero_fill(zf, blockIdx.x);
+    const int tid = threadIdx.x, T = blockDim.x;
     const int64_t row = (int64_t)blockIdx.x * K;
-    const int K4 = K >> 2;
-    float v[NV][4];
-    float ss = 0.0f;
+    const int K8 = K >> 3;
+    const bool mean = mode != BITNET_ACT_INT8_ABSMAX;
+    const bool nogain = gain == nullptr;
+    float v[NV8][8];
 #pragma unroll
-    for (int it = 0; it < NV; ++it) {
-        const int j = it * T + tid;
-        if (j < K4) {
-            src.get4(row + 4 * j, v[it]);
+    for (int it = 0; it < NV8; ++it) {
+        const int c = it * T + tid;
+        if (c < K8) {
+            src.get8(row + 8 * c, v[it]);
         } else {
-            v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.0f;
-        }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) ss = fmaf(v[it][e], v[it][e], ss);
-    }
-    ss = block_sum<T>(ss, red);
-    const float rn = rms_factor(ss, K, eps);
-
-    float part = 0.0f;
-#pragma unroll
-    for (int it = 0; it < NV; ++it) {
-        const int j = it * T + tid;
-        float g[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-        if (gain != nullptr && j < K4) {
-            const float4 gg = __ldg(reinterpret_cast<const float4 *>(gain) + j);
-            g[0] = gg.x; g[1] = gg.y; g[2] = gg.z; g[3] = gg.w;
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float y = __fmul_rn(v[it][e], rn);
-            if (gain != nullptr) y = __fmul_rn(y, g[e]);
-            v[it][e] = y;
-            part = mode == BITNET_ACT_INT8_ABSMAX ? fmaxf(part, fabsf(y)) : part + fabsf(y);
+            for (int e = 0; e < 8; ++e) v[it][e] = 0.0f;
         }
     }
-    float stat;
-    if (mode == BITNET_ACT_INT8_ABSMAX) {
-        stat = block_max<T>(part, red);
+    float ss = 0.0f, st = 0.0f;
+    if (mean) {
+#pragma unroll
+        for (int it = 0; it < NV8; ++it)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ss = fmaf(v[it][e], v[it][e], ss);
+                st += fabsf(v[it][e]);
+            }
     } else {
-        stat = __fdiv_rn(block_sum<T>(part, red), (float)K);
-    }
-    const QuantParams q = quant_params(stat, eps, mode);
 #pragma unroll
-    for (int it = 0; it < NV; ++it) {
-        const int j = it * T + tid;
-        if (j < K4) {
-            const uint32_t w = pack4(quant_byte(v[it][0], q.s, q.lo, q.hi), quant_byte(v[it][1], q.s, q.lo, q.hi),
-                                     quant_byte(v[it][2], q.s, q.lo, q.hi), quant_byte(v[it][3], q.s, q.lo, q.hi));
-            reinterpret_cast<uint32_t *>(codes + row)[j] = w;
+        for (int it = 0; it < NV8; ++it)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                ss = fmaf(v[it][e], v[it][e], ss);
+                st = fmaxf(st, fabsf(v[it][e]));
+            }
+    }
+    block_reduce2(ss, st, mean, red, [&](float2 r) {
+        ts.rn = rms_factor(r.x, K, eps);
+        if (nogain) {
+            const float ry = __fmul_rn(ts.rn, r.y);
+            ts.stat = mean ? __fdiv_rn(ry, (float)K) : ry;
+            const QuantParams q = quant_params(ts.stat, eps, mode);
+            ts.s = q.s;
+            ts.lo = q.lo;
+            ts.hi = q.hi;
+        }
+    });
+    const float rn = ts.rn;
+    if (nogain) {
+#pragma unroll
+        for (int it = 0; it < NV8; ++it)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[it][e] = __fmul_rn(v[it][e], rn);
+    } else {
+        float part = 0.0f;
+#pragma unroll
+        for (int it = 0; it < NV8; ++it) {
+            const int c = it * T + tid;
+            float g[8];
+            if (c < K8) {
+                const float4 g0 = __ldg(reinterpret_cast<const float4 *>(gain) + 2 * c);
+                const float4 g1 = __ldg(reinterpret_cast<const float4 *>(gain) + 2 * c + 1);
+                g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+                g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) g[e] = 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float y = __fmul_rn(__fmul_rn(v[it][e], rn), g[e]);
+                v[it][e] = y;
+                part = mean ? part + fabsf(y) : fmaxf(part, fabsf(y));
+            }
+        }
+        block_reduce2(0.0f, part, mean, red, [&](float2 r) {
+            ts.stat = mean ? __fdiv_rn(r.y, (float)K) : r.y;
+            const QuantParams q = quant_params(ts.stat, eps, mode);
+            ts.s = q.s;
+            ts.lo = q.lo;
+            ts.hi = q.hi;
+        });
+    }
+    const float qs = ts.s, qlo = ts.lo, qhi = ts.hi;
+    // int8: |y| <= gamma makes |y*s| < 127.5, so the clip can never act.
+#pragma unroll
+    for (int it = 0; it < NV8; ++it) {
+        const int c = it * T + tid;
+        if (c < K8) {
+            uint32_t f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = quant_bits(v[it][e], qs, qlo, qhi, mean);
+            *reinterpret_cast<uint2 *>(codes + row + 8 * c) =
+                make_uint2(pack4_perm(f[0], f[1], f[2], f[3]), pack4_perm(f[4], f[5], f[6], f[7]));
         }
     }
-    if (tid == 0) scale_x[blockIdx.x] = stat;
+    if (tid == 0) scale_x[blockIdx.x] = ts.stat;
 }
 
 // Launch with programmatic stream serialisation: the kernel may start while the
@@ -448,11 +524,10 @@ cudaError_t launch_fwht(const Src &src, int64_t M, const float *gain, float eps,
     return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, src, gain, eps, mode, codes, scale_x, zf);
 }
 
-template <int NV, class Src>
-cudaError_t launch_plain(const Src &src, int64_t M, int K, const float *gain, float eps, int mode,
+template <int NV8, class Src>
+cudaError_t launch_plain(const Src &src, int64_t M, int K, int T, const float *gain, float eps, int mode,
                          int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
-    constexpr int T = 256;
-    return launch_pdl(act_quant_plain_kernel<T, NV, Src>, dim3((unsigned)M), dim3(T), 0, s, src, gain, K, eps, mode,
+    return launch_pdl(act_quant_plain_kernel<NV8, Src>, dim3((unsigned)M), dim3(T), 0, s, src, gain, K, eps, mode,
                       codes, scale_x, zf);
 }
 
@@ -473,14 +548,20 @@ cudaError_t dispatch(const Src &src, int64_t M, int K, const float *gain, float 
             default: return cudaErrorInvalidValue;
         }
     }
-    const int nv = (int)ceil_div(K / 4, 256);
-    if (nv <= 1) return launch_plain<1>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 2) return launch_plain<2>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 4) return launch_plain<4>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 8) return launch_plain<8>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 16) return launch_plain<16>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    if (nv <= 32) return launch_plain<32>(src, M, K, gain, eps, mode, codes, scale_x, zf, s);
-    return cudaErrorInvalidValue;
+    // Few tokens (decode): about 256 threads per token, so each thread's serial work
+    // stays short.  Many tokens: 32 elements per thread (8 for short rows, 64 for
+    // K > 16384), so each CTA's per-token work is spread over more elements.  At most
+    // 512 threads.
+    const int k8 = K / 8;
+    int nv8;
+    if (M <= 64) nv8 = k8 <= 256 ? 1 : (k8 <= 512 ? 2 : (k8 <= 1024 ? 4 : 8));
+    else nv8 = k8 < 128 ? 1 : (k8 <= 2048 ? 4 : 8);
+    const int T = (int)ceil_div(ceil_div(k8, nv8), 32) * 32;
+    if (T > 512) return cudaErrorInvalidValue;
+    if (nv8 == 1) return launch_plain<1>(src, M, K, T, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv8 == 2) return launch_plain<2>(src, M, K, T, gain, eps, mode, codes, scale_x, zf, s);
+    if (nv8 == 4) return launch_plain<4>(src, M, K, T, gain, eps, mode, codes, scale_x, zf, s);
+    return launch_plain<8>(src, M, K, T, gain, eps, mode, codes, scale_x, zf, s);
 }
 
 }  // namespace
