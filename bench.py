@@ -213,9 +213,11 @@ def aggregate(elapsed_ms: float, tokens: float, world: int, backend_device=None)
 
 # ----------------------------------------------------------------------------- CPU oracle timing
 def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool = False):
-    """Time the oracle on a bounded sample of the workload.  Each case runs the full
-    per-token act_quant and the integer GEMM on a sample of output columns; the
-    time is extrapolated to all N columns.  Returns (tokens/s, description, steps)."""
+    """Time the oracle on a bounded sample of the workload.  Each case runs act_quant on
+    a sample of its tokens and the integer GEMM of those tokens on a sample of output
+    columns; the time is extrapolated to all M tokens and N columns.  The samples are
+    sized so that one step costs about budget_s / max(steps, 4) seconds.  Returns
+    (tokens/s, description, steps, seconds per step)."""
     import numpy as np
     from oracle import ref
     totals = []
@@ -226,28 +228,35 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
     for c in host:
         packed, alpha, _ = ref.pack_weights(c.W.numpy(), eps=c.eps)
         packs.append((packed, alpha))
-    # columns per case so one step costs about budget_s / max(steps, 4) seconds
     target_step = budget_s / max(4, steps or 4)
-    macs = sum(c.M * c.N * c.K for c in host)
-    mac_rate = 2.5e8  # rough single-core rate of the packed-weight loop, refined after the first step
-    frac = min(1.0, target_step * mac_rate / max(macs, 1))
+    elem_rate = 4e7   # rough single-core rate of the oracle's act_quant (elements/s)
+    mac_rate = 2.5e8  # rough single-core rate of the packed-weight loop (MAC/s)
+    row_frac = min(1.0, 0.5 * target_step * elem_rate / max(sum(c.M * c.K for c in host), 1))
+    rows = [max(1, min(c.M, int(math.ceil(c.M * row_frac)))) for c in host]
+    macs = sum(m * c.N * c.K for m, c in zip(rows, host))
+    frac = min(1.0, 0.5 * target_step * mac_rate / max(macs, 1))
+    # at least 8 columns, so that the call overhead stays small against the sampled work
+    cols = [max(min(c.N, 8), min(c.N, int(math.ceil(c.N * frac)))) for c in host]
+    # the dequant epilogue costs per output element: it runs on the full width of the
+    # sampled tokens (on zero sums), so only the integer GEMM is extrapolated over columns
+    acc_full = [np.zeros((m, c.N), np.int32) for m, c in zip(rows, host)]
     while True:
         t_step = 0.0
-        for c, (packed, alpha) in zip(host, packs):
+        for c, m, ncols, af, (packed, alpha) in zip(host, rows, cols, acc_full, packs):
             mode = ref.ACT_INT8 if c.mode == "int8" else ref.ACT_INT4
-            ncols = max(1, min(c.N, int(math.ceil(c.N * frac))))
-            X = c.X.float().numpy()
+            X = c.X[:m].float().numpy()
             t0 = time.perf_counter()
             if c.up is not None:
-                X = ref.swiglu(X, c.up.float().numpy())
-            q, s = ref.act_quant(X, None, c.eps, c.fwht, mode)
+                X = ref.swiglu(X, c.up[:m].float().numpy())
+            q, s_ = ref.act_quant(X, None, c.eps, c.fwht, mode)
             t1 = time.perf_counter()
-            acc = ref.gemm_packed(q, packed[:ncols], ncols)
-            o = ref.dequant(acc, s, alpha, mode)
+            ref.gemm_packed(q, packed[:ncols], ncols)
+            t2 = time.perf_counter()
+            o = ref.dequant(af, s_, alpha, mode)
             if bf16_out:
                 ref.round_bf16(o)
-            t2 = time.perf_counter()
-            t_step += (t1 - t0) + (t2 - t1) * (c.N / ncols)
+            t3 = time.perf_counter()
+            t_step += ((t1 - t0) + (t2 - t1) * (c.N / ncols) + (t3 - t2)) * (c.M / m)
         totals.append(t_step)
         done += 1
         elapsed = time.perf_counter() - t_begin
@@ -257,8 +266,11 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
             break
     tokens = sum(c.M for c in host)
     per_step = statistics.median(totals)
-    desc = (f"oracle (single-threaded C) on the same inputs: full act_quant per token, integer GEMM on "
-            f"{frac:.2%} of the output columns extrapolated to all N; {done} step(s), median")
+    sampled_rows = sum(rows)
+    desc = (f"oracle (single-threaded C) on the same inputs: act_quant on {sampled_rows} of {tokens} tokens, "
+            f"their integer GEMM on {sum(cols)} of {sum(c.N for c in host)} output columns, extrapolated to all "
+            f"tokens and columns; "
+            f"{done} step(s), median")
     return tokens / per_step, desc, done, per_step
 
 
