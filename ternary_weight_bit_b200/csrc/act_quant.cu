@@ -143,6 +143,11 @@ struct XSrc {
     const void *X;
     __device__ __forceinline__ void get8(int64_t idx, float *v) const { load8<BF16>(X, idx, v); }
     __device__ __forceinline__ void get4(int64_t idx, float *v) const { load4<BF16>(X, idx, v); }
+    // L2 prefetch of n elements from idx (a hint: it returns no data, so it is safe before
+    // the dependency wait -- L2 is where every write lands, so what is read later is current)
+    __device__ __forceinline__ void prefetch(int64_t idx, int n) const {
+        bulk_prefetch_l2(reinterpret_cast<const uint8_t *>(X) + idx * (BF16 ? 2 : 4), (uint32_t)n * (BF16 ? 2 : 4));
+    }
 };
 
 // silu(g) * u with silu(g) = g / (1 + e^-g), each step one IEEE rounding.
@@ -153,6 +158,10 @@ __device__ __forceinline__ float swiglu(float g, float u) {
 template <bool BF16>
 struct SwigluSrc {
     const void *gate, *up;
+    __device__ __forceinline__ void prefetch(int64_t idx, int n) const {
+        bulk_prefetch_l2(reinterpret_cast<const uint8_t *>(gate) + idx * (BF16 ? 2 : 4), (uint32_t)n * (BF16 ? 2 : 4));
+        bulk_prefetch_l2(reinterpret_cast<const uint8_t *>(up) + idx * (BF16 ? 2 : 4), (uint32_t)n * (BF16 ? 2 : 4));
+    }
     __device__ __forceinline__ void get8(int64_t idx, float *v) const {
         float u[8];
         load8<BF16>(gate, idx, v);
@@ -229,6 +238,7 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
     // may come from the previous kernel.  The GEMM waits for this kernel before it
     // reads the codes, so the order of the data is kept.
     pdl_launch_dependents();
+    if (threadIdx.x == 0) src.prefetch((int64_t)blockIdx.x * K, K);  // warm L2 while the producer finishes
     pdl_wait_prerequisites();
     zero_fill(zf, blockIdx.x);
 
@@ -386,6 +396,7 @@ act_quant_plain_kernel(Src src, const float *__restrict__ gain, int K, float eps
     __shared__ float2 red[32];
     __shared__ TokenScalars ts;
     pdl_launch_dependents();  // as in the FWHT kernel: the GEMM may launch, X is waited for
+    if (threadIdx.x == 0) src.prefetch((int64_t)blockIdx.x * K, K);  // warm L2 while the producer finishes
     pdl_wait_prerequisites();
     zero_fill(zf, blockIdx.x);
     const int tid = threadIdx.x, T = blockDim.x;
