@@ -805,6 +805,33 @@ def run_reference(args):
     print(json.dumps(result), flush=True)
 
 
+def run_library_int8_probe(args):
+    """Context only, not a bench line: the dense int8 GEMM rate torch._int_mm (cuBLASLt) reaches on
+    this GPU at 8192^3, beside the nominal-ratio int8 peak the roofline divides by."""
+    import torch
+    dev = torch.device("cuda", 0)
+    n = 8192
+    a = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-128, 128, (n, n), dtype=torch.int8, device=dev)
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = 20
+    e0.record()
+    for _ in range(reps):
+        torch._int_mm(a, b)
+    e1.record()
+    e1.synchronize()
+    s_ = e0.elapsed_time(e1) / 1e3 / reps
+    peaks, src = load_peaks()
+    print(json.dumps({"probe": "torch._int_mm int8 8192^3 (library GEMM, context)", "tops": round(2 * n ** 3 / s_ / 1e12, 1),
+                      "ms_per_gemm": round(s_ * 1e3, 3),
+                      "nominal_int8_peak_tops": round(2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 1),
+                      "peak_source": src}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -817,7 +844,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32",
                     help="output storage of the forward workloads: fp32, or bf16 rounded to nearest even")
+    ap.add_argument("--probe-library-int8", action="store_true",
+                    help="print the rate of torch._int_mm at 8192^3 (context for the int8 roofline) and exit")
     args = ap.parse_args()
+    if args.probe_library_int8:
+        run_library_int8_probe(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
