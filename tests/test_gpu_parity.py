@@ -513,6 +513,34 @@ def test_forward_deterministic_and_graph_capturable():
     assert torch.equal(out, o1)
 
 
+@pytest.mark.parametrize("M,fwht,mode", [(4, False, "int8"), (300, True, "int4"), (1, True, "int8")])
+def test_forward_chain_reads_the_previous_layers_output(M, fwht, mode):
+    # Three layers back to back on one stream, each reading the output the kernel just
+    # before it wrote (the GEMV/GEMM of the previous layer): the activation kernel may
+    # launch early and prefetch its input into L2, but reads it only after the
+    # dependency wait.  Each layer is checked against the oracle on the GPU's own input.
+    K = 1024
+    gen = synthetic.generator(M + 7)
+    X = synthetic.student_t3((M, K), gen)
+    Ws = [synthetic.gaussian((K, K), 0.02, gen) for _ in range(3)]
+    layers = [tb.HBitLinear(W.to(DEV), mode=mode, fwht=fwht) for W in Ws]
+    xs = [X.to(DEV)]
+    for layer in layers:
+        xs.append(layer(xs[-1]))
+    torch.cuda.synchronize()
+    for i, W in enumerate(Ws):
+        xin = host(xs[i]).astype(np.float32)
+        p_ref, a_ref, _ = ref.pack_weights(W.numpy(), eps=1e-5)
+        r = ref.hbitlinear_forward(xin, p_ref, a_ref, K, eps=1e-5, fwht_on=fwht, mode=MODES[mode])
+        codes, gs = tb.bitnet_act_quant(xs[i], eps=1e-5, fwht=fwht, mode=mode)
+        gcodes = host(codes)
+        sh = ref.shadow(xin, None, 1e-5, fwht, MODES[mode])
+        label = f"chain layer {i} M={M}"
+        parity.check_codes(gcodes, r.codes, sh, label)
+        same = ref.dequant(ref.gemm_packed(gcodes, p_ref, K), host(gs), a_ref, MODES[mode])
+        parity.check_out_same_codes(host(xs[i + 1]), same, label)
+
+
 def test_empty_batch_and_errors():
     W = synthetic.gaussian((64, 256), 0.02, synthetic.generator(1)).to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(W)
