@@ -281,20 +281,30 @@ BITNET_API bitnet_status_t bitnet_kv_quant(const void *kv, bitnet_dtype_t xdt, i
  * bitnet_forward_gemm_plan: the plan of the GEMM inside bitnet_hbitlinear_forward
  *   (and _noalloc) for the same problem: returns the token tile as above and writes
  *   the k-split count to *k_splits (if not NULL).  When the output has few tiles
- *   for the SMs, the forward splits K over up to 8 CTAs per tile: the partial int32
- *   sums are added with integer atomics (exact, order-independent) into `out`,
- *   which act_quant zeroes first, and the last split of each tile dequantises in
- *   place.  The result is bit-identical to the unsplit GEMM on the same codes.
+ *   for the SMs, the forward splits K over 2, 4 or 8 CTAs per tile.  Two halves:
+ *   the first to finish parks its int32 sums in the tile's own output rows and
+ *   raises a flag; the second (a CTA of the same grid, already running) waits for
+ *   the flag with a bounded wait, adds them and writes the result.  More splits:
+ *   the partial int32 sums are added with integer atomics (exact, order-
+ *   independent) into `out`, which act_quant zeroes first, and the last split of
+ *   each tile dequantises in place.  Either way the result is bit-identical to the
+ *   unsplit GEMM on the same codes.
  * bitnet_gemm_force_token_tile: process-wide override of that choice, for every
  *   device and thread: 0 restores the automatic choice; 256, 224, 192, 128 or 64
  *   forces it; any other value returns BITNET_ERR_INVALID_ARG and changes nothing.
  *   Results do not depend on the tile (the int32 accumulators are exact and the
  *   epilogue is elementwise), only the speed does.  For tests and tuning; set it
  *   while no other thread is launching GEMMs.
+ * bitnet_gemm_force_k_splits: the same kind of override for the forward's k-split
+ *   count: 0 restores the automatic choice; 1, 2, 4 or 8 forces it wherever the
+ *   shape allows that count (K/128 divisible by it, at least 4 k-blocks per split,
+ *   few enough tiles for the workspace counters); elsewhere the automatic choice
+ *   stands.  Any other value returns BITNET_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------ */
 BITNET_API int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K);
 BITNET_API int bitnet_forward_gemm_plan(int64_t M, int64_t N, int64_t K, int *k_splits);
 BITNET_API bitnet_status_t bitnet_gemm_force_token_tile(int token_tile);
+BITNET_API bitnet_status_t bitnet_gemm_force_k_splits(int k_splits);
 
 /* --------------------------------------------------------------------------
  * Status and diagnostics (no counterpart on the pages).

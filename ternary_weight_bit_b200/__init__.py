@@ -25,8 +25,10 @@ __all__ = [
     "BitnetError", "HBitLinear", "bitnet_pack_ternary", "bitnet_act_quant", "bitnet_ternary_gemm",
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
-    "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_forward_gemm_plan",
+    "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_gemm_force_k_splits",
+    "bitnet_forward_gemm_plan",
     "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu", "bitnet_kv_quant",
+    "bitnet_ternary_gemm_ex", "bitnet_hbitlinear_forward_ex",
 ]
 
 _MODES = {"int8": _native.ACT_INT8_ABSMAX, "int4": _native.ACT_INT4_ABSMEAN}
@@ -82,6 +84,11 @@ def bitnet_forward_gemm_plan(M: int, N: int, K: int) -> tuple:
 def bitnet_gemm_force_token_tile(token_tile: int) -> None:
     """Force the GEMM token tile (256/224/192/128/64) process-wide; 0 restores the automatic choice."""
     _native.check("bitnet_gemm_force_token_tile", _native.load().bitnet_gemm_force_token_tile(token_tile))
+
+
+def bitnet_gemm_force_k_splits(k_splits: int) -> None:
+    """Force the forward's k-split count (0 = automatic; 1, 2, 4, 8 where the shape allows it)."""
+    _native.check("bitnet_gemm_force_k_splits", _native.load().bitnet_gemm_force_k_splits(k_splits))
 
 
 def bitnet_pack_workspace_bytes(N: int, K: int) -> int:

@@ -73,6 +73,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_abi_version": (I, []),
         "bitnet_gemm_token_tile": (I, [I64, I64, I64]),
         "bitnet_gemm_force_token_tile": (I, [I]),
+        "bitnet_gemm_force_k_splits": (I, [I]),
         "bitnet_forward_gemm_plan": (I, [I64, I64, I64, ctypes.POINTER(ctypes.c_int)]),
     }
     for name, (res, args) in sigs.items():

@@ -215,13 +215,15 @@ __device__ __forceinline__ int reg_part(int p, int r) {
 __device__ __forceinline__ int pad(int i) { return i + (i >> 5); }
 
 // Zero the token's row of a following split-K GEMM's output (it adds int32 partial
-// sums there) and, in CTA 0, that GEMM's tile counters.  Runs after the dependency
+// sums there; a two-way split needs no zero rows) and, in CTA 0, that GEMM's tile
+// counters.  Runs after the dependency
 // wait: the buffers may still be read by earlier kernels until then.
 __device__ __forceinline__ void zero_fill(const ZeroFill &z, int64_t token) {
-    if (!z.rows) return;
-    uint32_t *row = z.rows + token * z.row_words;
-    for (int i = threadIdx.x; i < z.row_words; i += blockDim.x) row[i] = 0u;
-    if (token == 0)
+    if (z.rows) {
+        uint32_t *row = z.rows + token * z.row_words;
+        for (int i = threadIdx.x; i < z.row_words; i += blockDim.x) row[i] = 0u;
+    }
+    if (token == 0 && z.cnt)
         for (int i = threadIdx.x; i < z.cnt_n; i += blockDim.x) z.cnt[i] = 0;
 }
 

@@ -168,7 +168,10 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
     if (M > kGemvMaxM) {
         // a bf16 output cannot hold the int32 sums of a split GEMM: never split it
         plan = gemm_plan((int)M, (int)N, (int)K, sm_count(), out_bf16 ? 0 : kSplitCounters);
-        if (plan.splits > 1) {
+        if (plan.splits == 2) {
+            zf.cnt = tile_cnt;  // arrival counters and ready flags; the output needs no zeroing
+            zf.cnt_n = kSplitCounters;
+        } else if (plan.splits > 1) {
             zf.rows = reinterpret_cast<uint32_t *>(out);
             zf.row_words = (int)N;
             zf.cnt = tile_cnt;
@@ -341,6 +344,10 @@ int bitnet_forward_gemm_plan(int64_t M, int64_t N, int64_t K, int *k_splits) {
 
 bitnet_status_t bitnet_gemm_force_token_tile(int token_tile) {
     return gemm_force_tile(token_tile) ? BITNET_OK : BITNET_ERR_INVALID_ARG;
+}
+
+bitnet_status_t bitnet_gemm_force_k_splits(int k_splits) {
+    return gemm_force_splits(k_splits) ? BITNET_OK : BITNET_ERR_INVALID_ARG;
 }
 
 bitnet_status_t bitnet_kv_quant(const void *kv, bitnet_dtype_t xdt, int64_t BH, int64_t S, int64_t D, int bits,

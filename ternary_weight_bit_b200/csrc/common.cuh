@@ -33,6 +33,32 @@ __device__ __forceinline__ void record_timeout(int *status) {
     if (status) atomicCAS(status, 0, (int)BITNET_ERR_TIMEOUT);
 }
 
+// ---------------------------------------------------------------- flags between CTAs
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until *flag != 0 (set by another CTA of the same grid, which is running: it
+// has already taken its turn).  Returns false (and records BITNET_ERR_TIMEOUT) if the
+// limit passes first.
+__device__ __forceinline__ bool flag_wait_set(const int *flag, int *status, uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_gpu(flag) != 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i) {
+            if (ld_acquire_gpu(flag) != 0) return true;
+            __nanosleep(64);
+        }
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_timeout(status);
+            return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

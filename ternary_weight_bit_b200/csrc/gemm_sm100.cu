@@ -343,7 +343,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
             if (!mbar_wait_u32(ACCFULL + 8 * b, (uint32_t)(tc / DB) & 1u, status)) break;
             tc_fence_after();
             const int n = n0 + r;
-            if (splits > 1) {
+            // Pair split (two halves of K): the first half to finish parks its int32 sums
+            // in the tile's own output rows, the second adds them and writes the result.
+            bool pair_first = false, pair_second = false;
+            if (splits == 2) {
+                if (et == 0) s_last = atomicAdd(tile_cnt + tile, 1);  // 0: first, 1: second
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                pair_second = s_last != 0;
+                pair_first = !pair_second;
+                if (pair_second) {
+                    if (et == 0) flag_wait_set(tile_cnt + kPairFlags + tile, status);
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    __threadfence();
+                }
+            } else if (splits > 1) {
                 // Add this split's partial sums to the int32 image of the tile (integer
                 // atomics: the total does not depend on their order).
 #pragma unroll 1
@@ -399,6 +412,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_base + lane_off + (uint32_t)(b * BT + 32 * c), v);
                 tmem_wait_ld();
+                if (splits == 2) {
+                    // A whole 32-token chunk of a full-width tile is parked in a coalesced
+                    // order: row r's 32 sums fill 128 contiguous bytes of token row
+                    // m0 + 32c + r/4 at column n0 + 32 (r % 4).  Ragged chunks keep the
+                    // natural [token][row] order.
+                    const bool whole = m0 + 32 * c + 32 <= M && n0 + BW <= N && (N & 3) == 0;
+                    int32_t *seg = acc_img + (int64_t)(m0 + 32 * c + (r >> 2)) * N + n0 + 32 * (r & 3);
+                    if (pair_first) {
+                        if (whole) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4)
+                                *reinterpret_cast<int4 *>(seg + 4 * q4) =
+                                    make_int4((int)v[4 * q4], (int)v[4 * q4 + 1], (int)v[4 * q4 + 2], (int)v[4 * q4 + 3]);
+                        } else if (n < N) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int m = m0 + 32 * c + j;
+                                if (m < M) acc_img[(int64_t)m * N + n] = (int)v[j];
+                            }
+                        }
+                        continue;  // the second half writes the output
+                    }
+                    if (whole) {
+                        int4 pq[8];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) pq[q4] = __ldcg(reinterpret_cast<const int4 *>(seg + 4 * q4));
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            v[4 * q4] = (uint32_t)((int)v[4 * q4] + pq[q4].x);
+                            v[4 * q4 + 1] = (uint32_t)((int)v[4 * q4 + 1] + pq[q4].y);
+                            v[4 * q4 + 2] = (uint32_t)((int)v[4 * q4 + 2] + pq[q4].z);
+                            v[4 * q4 + 3] = (uint32_t)((int)v[4 * q4 + 3] + pq[q4].w);
+                        }
+                    } else if (n < N) {
+                        int32_t pq[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int m = m0 + 32 * c + j;
+                            pq[j] = m < M ? __ldcg(acc_img + (int64_t)m * N + n) : 0;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = (uint32_t)((int)v[j] + pq[j]);
+                    }
+                    // every thread's reads of the parked sums are done before any output
+                    // of this chunk replaces them
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                }
                 if (tma_out) {
                     // [32 tokens][128 rows] through shared memory, one bulk tensor store
                     const int buf = ck & 1;
@@ -443,6 +503,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars + 2 * ST + 2 * AS + DB + b);  // the buffer may be overwritten
+            if (pair_first) {
+                __threadfence();  // this thread's parked sums are visible before the flag below
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (et == 0) atomicExch(tile_cnt + kPairFlags + tile, 1);
+            } else if (pair_second && et == 0) {
+                tile_cnt[tile] = 0;  // ready for the next call
+                tile_cnt[kPairFlags + tile] = 0;
+            }
             asm volatile("bar.sync 1, 128;" ::: "memory");              // fac row b is rewritten DB tiles later
         }
         if (et == 0 && tma_out) bulk_wait_group<0>();  // the last stores have landed
@@ -468,7 +536,7 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
     // The bulk-store epilogue needs a 16-byte row pitch and base, and a box that fits.
     memset(&to, 0, sizeof(to));
     // (N elements of 4 or 2 bytes per row: N % 4 == 0 for fp32, N % 8 == 0 for bf16)
-    const bool store_ok = splits == 1 && N % (out_bf16 ? 8 : 4) == 0 && M >= OUT_TOKENS && N >= BW &&
+    const bool store_ok = splits <= 2 && N % (out_bf16 ? 8 : 4) == 0 && M >= OUT_TOKENS && N >= BW &&
                           (reinterpret_cast<uintptr_t>(out) & 15) == 0;
     const int tma_out =
         store_ok && make_tmap_out_2d(&to, out, out_bf16, (uint64_t)N, (uint64_t)M, BW, OUT_TOKENS) ? 1 : 0;
@@ -502,28 +570,35 @@ cudaError_t launch_cfg(const int8_t *codes, const float *scale_x, int mode, cons
 
 // Modelled time of a (token tile, k-split) choice, in units of one 128-k stage of one
 // tile: rounds of work units per SM x (stages per unit x relative stage cost + a
-// drain stall per unit when the accumulator is single-buffered + the split-K
-// epilogue).  All constants are B200 measurements: a stage takes about as long at
-// 192..256 tokens; the single-buffered 256-token tile stalls about 10 stages per
-// tile; a split tile costs about 20 + BT/4 stages more (the atomic additions, and
-// the last split dequantising the whole tile), so splitting only pays for few
-// output tiles and long K.
+// drain stall per unit when the accumulator is single-buffered + the split fixup).
+// All constants are B200 measurements: a stage takes about as long at 192..256
+// tokens; the single-buffered 256-token tile stalls about 10 stages per tile; a tile
+// split in two costs about 5 BT / 16 stages more (the first half parks its sums, the
+// second reads them back chunk by chunk), one split further with atomics about
+// 20 + BT / 4, so splitting only pays for few output tiles and long K.
 double gemm_tile_cost(int bt, int splits, int M, int N, int K, int sms) {
     const double w = bt >= 192 ? 1.0 : (bt >= 128 ? 0.93 : 0.81);
     const double drain = bt == 256 ? 10.0 : 0.0;
-    const double split_cost = splits == 1 ? 0.0 : 20.0 + bt / 4.0;
+    const double split_cost = splits == 1 ? 0.0 : (splits == 2 ? bt * 5.0 / 16.0 : 20.0 + bt / 4.0);
     const long units = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt) * splits;
     const long rounds = (units + sms - 1) / sms;
     return (double)rounds * ((double)(K / BK / splits) * w + drain + split_cost);
 }
 
 namespace {
-int g_forced_tile = 0;  // 0: automatic
+int g_forced_tile = 0;    // 0: automatic
+int g_forced_splits = 0;  // 0: automatic
 }  // namespace
 
 bool gemm_force_tile(int bt) {
     if (bt != 0 && bt != 256 && bt != 224 && bt != 192 && bt != 128 && bt != 64) return false;
     g_forced_tile = bt;
+    return true;
+}
+
+bool gemm_force_splits(int splits) {
+    if (splits != 0 && splits != 1 && splits != 2 && splits != 4 && splits != 8) return false;
+    g_forced_splits = splits;
     return true;
 }
 
@@ -537,7 +612,10 @@ GemmPlan gemm_plan(int M, int N, int K, int sms, int max_split_tiles) {
         if (g_forced_tile && bt != g_forced_tile) continue;
         const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
         for (int sp : splits_c) {
+            // a forced count applies where splitting is allowed at all (the forward)
+            if (g_forced_splits && max_split_tiles > 0 && sp != g_forced_splits) continue;
             if (sp > 1 && (tiles > max_split_tiles || KB % sp != 0 || KB / sp < 4)) continue;
+            if (sp == 2 && tiles > kPairFlags) continue;  // arrival counters and flags share the workspace
             const double c = gemm_tile_cost(bt, sp, M, N, K, sms);
             if (c < best_cost * 0.999) {
                 best = GemmPlan{bt, sp};

@@ -59,15 +59,21 @@ cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, con
 
 // Prefill path: tcgen05 int8 tensor-core GEMM with TMEM accumulators.
 // A plan is a token-tile size (256/224/192/128/64) and a k-split count (1, 2, 4, 8).
-// With splits > 1, `out` must be zero on entry (the kernel adds int32 partial sums
-// into it before dequantising in place) and tile_cnt must point at
-// kSplitCounters zeroed ints (the kernel leaves them zero again).  A bf16 output
+// With splits > 2, `out` must be zero on entry (the kernel adds int32 partial sums
+// into it before dequantising in place); with splits == 2 it needs no zeroing (the
+// pair split below).  With splits > 1, tile_cnt must point at kSplitCounters zeroed
+// ints (the kernel leaves them zero again).  A bf16 output
 // (out_bf16) is never split.
 struct GemmPlan {
     int token_tile;  // 0: choose automatically (no split)
     int splits;
 };
 constexpr int kSplitCounters = 1024;
+// A two-way split ("pair split") keeps per tile an arrival counter (int tile) and a
+// ready flag (int kPairFlags + tile) in the same workspace, so it serves up to
+// kPairFlags tiles.  The first half to finish parks its int32 sums in the tile's own
+// output rows; `out` needs no zeroing then, only the counters.
+constexpr int kPairFlags = kSplitCounters / 2;
 cudaError_t launch_gemm_tc(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                            const float *alpha, int M, int N, int K, void *out, int32_t *acc_out,
                            bool pdl, cudaStream_t s, GemmPlan plan = GemmPlan{0, 1}, int *tile_cnt = nullptr,
@@ -81,6 +87,9 @@ int gemm_pick_tile(int M, int N, int K, int sms);
 double gemm_tile_cost(int bt, int splits, int M, int N, int K, int sms);
 // Force the token tile (0 = automatic); false for an unsupported value.
 bool gemm_force_tile(int bt);
+// Force the forward's k-split count (0 = automatic; 1, 2, 4 or 8) where the shape
+// allows it; false for an unsupported value.
+bool gemm_force_splits(int splits);
 
 // The forward's kernels (act_quant, then GEMV or GEMM), arguments validated;
 // tile_cnt points at kSplitCounters ints of workspace for a split-K GEMM.  With

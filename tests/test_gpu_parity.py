@@ -345,7 +345,7 @@ def test_forward_ragged(M, K, N, mode, fwht, xdt):
 def _split_k_case(M, K, N, mode, fwht, seed):
     case = synthetic.make_case("splitk", M, K, N, x_kind="student_t3", outliers=max(1, K // 100), outlier_gain=50.0,
                                x_dtype="f32", fwht=fwht, mode=mode, seed=seed)
-    _forward_case(case)  # against the oracle
+    _forward_case(case, None if M < 200 else _sample(M, 24))  # against the oracle
     # bit-identical to the unsplit GEMM on the same codes
     Xd = case.X.to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(case.W.to(DEV), eps=case.eps)
@@ -358,14 +358,31 @@ def _split_k_case(M, K, N, mode, fwht, seed):
 
 @pytest.mark.parametrize("M,K,N,mode,fwht,splits", [
     (40, 16384, 1000, "int8", False, 8),  # ragged tokens and weight rows
-    (33, 8192, 4096, "int4", True, 4),
+    (33, 8192, 4096, "int4", True, 2),
     (64, 16384, 2048, "int8", False, 8),
-    (128, 8192, 2048, "int4", True, 4),
+    (128, 8192, 2048, "int4", True, 2),
+    (200, 8192, 1000, "int8", False, 2),   # pair split: ragged tokens and weight rows
+    (300, 8192, 998, "int4", True, 2),     # pair split, N % 4 != 0 (direct stores)
+    (260, 16384, 2000, "int4", True, 2),   # pair split, 128-token tiles
 ])
 def test_forward_split_k(M, K, N, mode, fwht, splits):
-    # few output tiles for the SMs: the forward splits K (int32 atomics into out)
+    # few output tiles for the SMs: the forward splits K.  Two halves: the first parks
+    # its int32 sums in the tile's output rows and the second adds them; more splits
+    # add int32 partial sums into a zeroed output with atomics.
     assert tb.bitnet_forward_gemm_plan(M, N, K)[1] == splits
     _split_k_case(M, K, N, mode, fwht, seed=M * 7 + K)
+
+
+@pytest.mark.parametrize("splits", [2, 4, 8])
+def test_forward_forced_k_splits(splits):
+    # every split protocol on the M = 512 sweep shape, whose automatic plan does not
+    # split (whole 256-token chunks for the pair split), bit-identical to the unsplit GEMM
+    try:
+        tb.bitnet_gemm_force_k_splits(splits)
+        assert tb.bitnet_forward_gemm_plan(512, 4096, 16384)[1] == splits
+        _split_k_case(512, 16384, 4096, "int4", True, seed=splits)
+    finally:
+        tb.bitnet_gemm_force_k_splits(0)
 
 
 @pytest.mark.parametrize("tile", [256, 224, 192, 128, 64])
