@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 5
+#define BITNET_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))

@@ -608,18 +608,21 @@ GemmPlan gemm_plan(int M, int N, int K, int sms, int max_split_tiles) {
     GemmPlan best{256, 1};
     double best_cost = 1e300;
     const int KB = K / BK;
-    for (int bt : tiles_c) {
-        if (g_forced_tile && bt != g_forced_tile) continue;
-        const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
-        for (int sp : splits_c) {
-            // a forced count applies where splitting is allowed at all (the forward)
-            if (g_forced_splits && max_split_tiles > 0 && sp != g_forced_splits) continue;
-            if (sp > 1 && (tiles > max_split_tiles || KB % sp != 0 || KB / sp < 4)) continue;
-            if (sp == 2 && tiles > kPairFlags) continue;  // arrival counters and flags share the workspace
-            const double c = gemm_tile_cost(bt, sp, M, N, K, sms);
-            if (c < best_cost * 0.999) {
-                best = GemmPlan{bt, sp};
-                best_cost = c;
+    // a forced split count applies where splitting is allowed at all (the forward) and
+    // the shape admits it; otherwise the automatic choice stands
+    for (int pass = (g_forced_splits && max_split_tiles > 0) ? 0 : 1; pass < 2 && best_cost == 1e300; ++pass) {
+        for (int bt : tiles_c) {
+            if (g_forced_tile && bt != g_forced_tile) continue;
+            const long tiles = (long)((N + BW - 1) / BW) * ((M + bt - 1) / bt);
+            for (int sp : splits_c) {
+                if (pass == 0 && sp != g_forced_splits) continue;
+                if (sp > 1 && (tiles > max_split_tiles || KB % sp != 0 || KB / sp < 4)) continue;
+                if (sp == 2 && tiles > kPairFlags) continue;  // arrival counters and flags share the workspace
+                const double c = gemm_tile_cost(bt, sp, M, N, K, sms);
+                if (c < best_cost * 0.999) {
+                    best = GemmPlan{bt, sp};
+                    best_cost = c;
+                }
             }
         }
     }

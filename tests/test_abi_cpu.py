@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 5
+    assert L.bitnet_abi_version() == 6
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
@@ -51,6 +51,33 @@ def test_gemm_token_tile_host_logic(L):
             assert L.bitnet_gemm_token_tile(4096, 4096, 4096) == good  # a forced tile wins
     finally:
         assert L.bitnet_gemm_force_token_tile(0) == _native.OK
+
+
+def test_forward_split_plans(L):
+    # the forward's (token tile, k-split) plans for the sweep shapes on a 148-SM B200
+    # (the host answers without a GPU): two halves at 128-256 tokens of long K, four
+    # atomic splits at 64 tokens, no split at 512 (measured faster unsplit)
+    def plan(M, N, K):
+        sp = ctypes.c_int(-1)
+        bt = L.bitnet_forward_gemm_plan(M, N, K, ctypes.byref(sp))
+        return bt, sp.value
+    assert plan(256, 4096, 16384) == (128, 2)
+    assert plan(128, 2048, 8192) == (64, 2)
+    assert plan(64, 4096, 16384) == (64, 4)
+    assert plan(512, 4096, 16384) == (128, 1)
+    assert plan(4096, 4096, 4096) == (224, 1)
+    for bad in (3, 5, 16, -1):
+        assert L.bitnet_gemm_force_k_splits(bad) == _native.ERR_INVALID_ARG
+    try:
+        for forced in (1, 2, 4, 8):
+            assert L.bitnet_gemm_force_k_splits(forced) == _native.OK
+            assert plan(512, 4096, 16384)[1] == forced
+        assert L.bitnet_gemm_force_k_splits(8) == _native.OK
+        # 8 k-blocks: a split needs at least 4 per part, so the automatic plan stands
+        assert plan(64, 4096, 1024) == (64, 1)
+    finally:
+        assert L.bitnet_gemm_force_k_splits(0) == _native.OK
+    assert L.bitnet_gemm_token_tile(512, 4096, 16384) == 128  # the standalone GEMM never splits
 
 
 def test_kv_quant_validation(L):
