@@ -18,7 +18,16 @@ With N > 1 (torchrun), every rank runs its own replica of the workload (the path
 has no cross-GPU exchange); value = tokens of all ranks / max rank time.
 
 --impl reference times the CPU oracle (single-threaded C, test infrastructure)
-on the same workload, on rank 0 only.
+on the same workload, on rank 0 only, each step a bounded sample of tokens and
+output columns extrapolated to the whole step.
+
+Other workloads (--workload): prefill, wdown, wdown_swiglu, msweep_M<M>, kvcache.
+--out-dtype bf16 stores the forward workloads' outputs in bf16.  Besides the
+contract's keys the line carries `roofline` (the dominant kernel alone, timed in one
+graph over every input rotation), `act_quant` (the activation kernel alone, the same
+way), `e2e` (the public forward with pinned host buffers in and out) and `clocks`.
+--probe-library-int8 prints cuBLASLt's dense int8 GEMM rate at 8192^3 instead, for
+context beside the int8 roofline.
 """
 from __future__ import annotations
 
