@@ -21,7 +21,9 @@
  *     synchronising; results are ready when the stream reaches them.  The kernels
  *     use programmatic dependent launch: they may begin while the previous kernel on
  *     the stream finishes.  Before their dependency wait they read only the packed
- *     weights (prefetch and first loads); every other input is read after it.  So
+ *     weights (the decode kernel's first loads); they may also issue L2 prefetches
+ *     of their other inputs, hints that return no data.  Every other input is read
+ *     after the wait.  So
  *     `packed` must not be written by the kernel immediately preceding a call on its
  *     stream, unless that kernel is bitnet_pack_ternary's (it fences its stores) or
  *     ends every writing thread with __threadfence(); copies, events, other streams
