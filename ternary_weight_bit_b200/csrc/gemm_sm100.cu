@@ -32,6 +32,13 @@
 //                owns TMEM lanes 32 (w % 4) .. +31 (= weight rows) of its slot.
 //   4 epilogue warps: tcgen05.ld, out[m][n] = acc * f[m]; the fp32 (or bf16) tile goes
 //                out through shared memory with one TMA bulk tensor store per 32 tokens.
+//
+// Split K (forward only, few output tiles): a work unit is (tile, split).  Two
+// splits: the first to finish parks its int32 sums in the tile's output rows and
+// raises a flag; the second, a CTA of this persistent grid, waits for the flag, adds
+// and writes the output.  Four or eight: every split adds its sums into the zeroed
+// output with integer atomics and the last one (per a tile counter) dequantises in
+// place.  Both are exact, so the result equals the unsplit GEMM bit for bit.
 // All waits are bounded; a timeout is recorded in the device status word.
 #include <string.h>
 
