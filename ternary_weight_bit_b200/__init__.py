@@ -344,7 +344,9 @@ class HBitLinear:
     """Pack once, forward many: an H-BitLinear layer over a fixed weight matrix.
 
     W is [out_features, in_features] fp32 on a CUDA device.  fwht=True gives the
-    H-BitLinear of the BitNet v2 page (Wo / Wdown); fwht=False the plain BitLinear."""
+    H-BitLinear of the BitNet v2 page (Wo / Wdown); fwht=False the plain BitLinear.
+    The layer keeps one forward workspace and reuses it, so calls of the same layer
+    on different streams must be ordered (events, or one stream)."""
 
     def __init__(self, W: torch.Tensor, mode="int8", fwht: bool = True, eps: float = 1e-5, gain=None):
         self.N, self.K = W.shape
