@@ -488,3 +488,33 @@ def test_bf16_is_odd_and_monotone():
     np.testing.assert_array_equal(ref.round_bf16(-x), b ^ np.uint16(0x8000))
     v = _bf16_value(b.astype(np.uint32)).view(np.float32)
     assert (np.diff(v) >= 0).all()
+
+
+# ----------------------------------------------------------------------------- the rotation's purpose
+# (bitnet_v2_engine.py page: the Hadamard step spreads outlier channels so that the
+# activation distribution becomes closer to Gaussian before the low-bit quantiser)
+def test_fwht_gaussianises_heavy_tailed_tokens():
+    from ternary_weight_bit_b200 import synthetic
+    gen = synthetic.generator(31)
+    K = 8192
+    X = synthetic.student_t3((6, K), gen)
+    X[:, synthetic.outlier_channels(K, 82, gen)] *= 50.0  # the wdown input: 1 % channels x50
+    x = ref.rmsnorm(X.numpy())
+    y = ref.fwht(x)
+
+    def excess_kurtosis(a):
+        a = a.astype(np.float64)
+        m = a.mean(axis=1, keepdims=True)
+        v = ((a - m) ** 2).mean(axis=1)
+        return ((a - m) ** 4).mean(axis=1) / v ** 2 - 3.0
+
+    def peak_to_rms(a):
+        a = a.astype(np.float64)
+        return np.abs(a).max(axis=1) / np.sqrt((a * a).mean(axis=1))
+
+    kx, ky = excess_kurtosis(x), excess_kurtosis(y)
+    px, py = peak_to_rms(x), peak_to_rms(y)
+    assert (kx > 20).all() and (np.abs(ky) < 0.5).all()  # heavy-tailed in, close to Gaussian out
+    assert (px > 5 * py).all() and (py < 6).all()       # the outliers are spread over all channels
+    # the transform is orthogonal: the mean square (RMSNorm made it 1) is kept
+    np.testing.assert_allclose((y.astype(np.float64) ** 2).mean(axis=1), 1.0, rtol=1e-4)
