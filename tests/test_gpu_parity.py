@@ -558,6 +558,55 @@ def test_forward_chain_reads_the_previous_layers_output(M, fwht, mode):
         parity.check_out_same_codes(host(xs[i + 1]), same, label)
 
 
+def _guarded(n, dtype, poison, pad):
+    """A flat buffer of pad + n + pad elements filled with `poison`; returns it and the
+    middle n elements (16-byte aligned when pad is a multiple of 16 bytes)."""
+    big = torch.full((pad + n + pad,), poison, dtype=dtype, device=DEV)
+    return big, big[pad:pad + n]
+
+
+@pytest.mark.parametrize("M,K,N,mode,fwht,out_dt", [
+    (5, 2560, 700, "int8", False, torch.float32),    # decode kernel, ragged N
+    (77, 384, 130, "int4", False, torch.float32),    # GEMM, direct stores (M < 32 tokens per box)
+    (300, 8192, 998, "int4", True, torch.float32),   # pair split, N % 4 != 0
+    (200, 8192, 1000, "int8", False, torch.float32), # pair split, ragged tiles
+    (40, 16384, 1000, "int8", False, torch.float32), # atomic split, ragged
+    (2000, 384, 2600, "int8", False, torch.float32), # GEMM, bulk-store epilogue
+    (64, 256, 1990, "int4", False, torch.bfloat16),  # bf16 output, N % 8 != 0
+    (130, 1024, 2048, "int8", True, torch.bfloat16), # bf16 output, bulk-store epilogue
+])
+def test_writes_stay_inside_the_output_and_workspace(M, K, N, mode, fwht, out_dt):
+    # guard bands around the output and the workspace: every byte outside them must
+    # keep its poison after the forward
+    gen = synthetic.generator(M + N)
+    X = synthetic.student_t3((M, K), gen).to(DEV)
+    W = synthetic.gaussian((N, K), 0.02, gen).to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(W)
+    pad = 4096  # elements of the output: 8 or 16 KB, 16-byte aligned either way
+    poison = -7777.0
+    obig, out_flat = _guarded(M * N, out_dt, poison, pad)
+    out = out_flat.view(M, N)
+    nbytes = tb.bitnet_forward_workspace_bytes(M, K)
+    wpad = 4096  # bytes, a multiple of 256
+    wbig, ws = _guarded(nbytes, torch.uint8, 0xA5, wpad)
+    if out_dt == torch.float32:
+        tb.bitnet_hbitlinear_forward(X, packed, alpha, N, fwht=fwht, mode=mode, out=out, ws=ws)
+    else:
+        tb.bitnet_hbitlinear_forward_ex(X, packed, alpha, N, fwht=fwht, mode=mode, out_dtype=out_dt, out=out, ws=ws)
+    torch.cuda.synchronize()
+    assert tb.bitnet_get_last_device_status() == 0
+    ob = obig.float().cpu()
+    stored = torch.full((1,), poison, dtype=out_dt).float().item()  # the poison as the dtype holds it
+    assert bool((ob[:pad] == stored).all()) and bool((ob[pad + M * N:] == stored).all()), "write outside the output"
+    assert bool(torch.isfinite(ob[pad:pad + M * N]).all())
+    wb = wbig.cpu()
+    assert bool((wb[:wpad] == 0xA5).all()) and bool((wb[wpad + nbytes:] == 0xA5).all()), "write outside the workspace"
+    # and the result is the unguarded forward's
+    ref_out = (tb.bitnet_hbitlinear_forward(X, packed, alpha, N, fwht=fwht, mode=mode) if out_dt == torch.float32 else
+               tb.bitnet_hbitlinear_forward_ex(X, packed, alpha, N, fwht=fwht, mode=mode, out_dtype=out_dt))
+    assert torch.equal(out, ref_out)
+
+
 def test_empty_batch_and_errors():
     W = synthetic.gaussian((64, 256), 0.02, synthetic.generator(1)).to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(W)
