@@ -28,7 +28,7 @@ ACT_INT4_ABSMEAN = 1
 F32 = 0
 BF16 = 1
 
-_LIB = None
+_LIBS: dict = {}  # loaded libraries by path
 
 
 class BitnetError(RuntimeError):
@@ -46,9 +46,8 @@ def declared_symbols(header: str = HEADER) -> list[str]:
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     """Load libbitnet.so and declare its signatures (no CUDA call is made)."""
-    global _LIB
-    if _LIB is not None:
-        return _LIB
+    if path in _LIBS:
+        return _LIBS[path]
     if not os.path.exists(path):
         raise RuntimeError(f"libbitnet.so not built: {path} is missing (run __graft_entry__.build())")
     L = ctypes.CDLL(path)
@@ -80,7 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
-    _LIB = L
+    _LIBS[path] = L
     return L
 
 

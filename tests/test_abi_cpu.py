@@ -162,3 +162,22 @@ def test_empty_batch_is_a_noop(L):
     assert L.bitnet_ternary_gemm(None, None, 0, None, None, 0, 16, 256, None, None, s) == _native.OK
     assert L.bitnet_hbitlinear_forward(None, 0, 0, 256, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, None, 0,
                                        s) == _native.OK
+
+
+def test_no_cpu_fallback():
+    # the product path refuses host tensors instead of computing anything on the CPU
+    import pytest
+    import torch
+    import ternary_weight_bit_b200 as tb
+    X = torch.randn(4, 256)
+    W = torch.randn(64, 256)
+    with pytest.raises(ValueError, match="CUDA"):
+        tb.bitnet_pack_ternary(W)
+    with pytest.raises(ValueError, match="CUDA"):
+        tb.bitnet_act_quant(X)
+    with pytest.raises(ValueError, match="CUDA"):
+        tb.bitnet_hbitlinear_forward(X, torch.zeros(64, 64, dtype=torch.uint8), torch.ones(1), 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        tb.bitnet_kv_quant(torch.randn(1, 2, 3, 64))
+    with pytest.raises(RuntimeError, match="not built"):
+        _native.load("/nonexistent/libbitnet.so")
