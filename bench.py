@@ -1,31 +1,38 @@
 #!/usr/bin/env python3
 """Benchmark of the B200 H-BitLinear forward path (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload decode|...]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 A step is one pass of the whole per-token path -- RMSNorm, optional FWHT,
 activation quantisation, ternary GEMM/GEMV, fp32 epilogue -- over one batch of
 the workload (weights are packed once, before timing, as a deployment would).
-The default workload is the decode GEMV configuration: int8 absmax, no FWHT,
-M in {1, 4, 8} tokens against W [6912 x 2560] and the transposed W [2560 x 6912];
-one step runs the six forwards.  Inputs are seeded synthetic tensors.
+The default workload is the largest configuration that fits one GPU: the M = 8192
+point of the 4096-hidden M-sweep, int4 absmean + FWHT, X Student-t(3) with 1 %
+outlier channels x50, against Wo [4096 x 4096] and Wdown [4096 x 16384]; one step
+runs the two forwards (1.37 Tera integer ops).  The same line carries a `decode`
+sub-record: the decode configuration (int8 absmax, no FWHT, M in {1, 4, 8} against
+W [6912 x 2560] and [2560 x 6912], six forwards per step) measured the same way with
+its own roofline, step time and CPU baseline.  Inputs are seeded synthetic tensors.
 
 Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
 bracketed by a barrier and a device synchronisation, timed with CUDA events on the
-launching stream; the maximum over ranks is reported.  The packed weights rotate
-over enough copies that every step reads them from HBM (total > 4x L2).
-With N > 1 (torchrun), every rank runs its own replica of the workload (the path
-has no cross-GPU exchange); value = tokens of all ranks / max rank time.
+launching stream; the maximum over ranks is reported.  Inputs larger than 4x L2
+(the default workload's step reads 691 MiB), or rotated over enough copies that
+every step reads them from HBM.  Clocks are read through NVML every 2 ms during the
+timed region.  With N > 1 (torchrun), every rank runs its own replica of the
+workload (the path has no cross-GPU exchange); value = tokens of all ranks / max
+rank time.
 
 --impl reference times the CPU oracle (single-threaded C, test infrastructure)
 on the same workload, on rank 0 only, each step a bounded sample of tokens and
 output columns extrapolated to the whole step.
 
-Other workloads (--workload): prefill, wdown, wdown_swiglu, msweep_M<M>, kvcache.
---out-dtype bf16 stores the forward workloads' outputs in bf16.  Besides the
-contract's keys the line carries `roofline` (the dominant kernel alone, timed in one
-graph over every input rotation), `act_quant` (the activation kernel alone, the same
-way), `e2e` (the public forward with pinned host buffers in and out) and `clocks`.
+Other workloads (--workload): decode, prefill, wdown, wdown_swiglu, msweep_M<M>,
+kvcache.  --out-dtype bf16 stores the forward workloads' outputs in bf16.  Besides
+the contract's keys the line carries `roofline` (the dominant kernel alone, timed in
+one graph over every input rotation), `act_quant` (the activation kernel alone, the
+same way), `e2e`
+(the public forward with pinned host buffers in and out) and `clocks`.
 --probe-library-int8 prints cuBLASLt's dense int8 GEMM rate at 8192^3 instead, for
 context beside the int8 roofline.
 """
@@ -47,6 +54,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ternary GEMM TOPS & weight GB/s vs roofline; H-BitLinear tokens/s (1 B200)"
+# The largest configuration that fits one GPU: the M = 8192 point of the 4096-hidden
+# M-sweep (Wo [4096 x 4096] and Wdown [4096 x 16384], int4 + FWHT), 1.37 Tera int ops
+# per step.  The default run adds the decode configuration as a sub-record.
+DEFAULT_WORKLOAD = "msweep_M8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -91,6 +102,11 @@ def workload_text(name):
         return WORKLOAD_TEXT[name]
     return f"M-sweep point ({name}): int4 + FWHT, Student-t(3) X with 1% outlier channels x50; Wo [4096x4096] " \
            f"and Wdown [4096x16384]"
+
+
+def _xdt_name(c):
+    """"bf16" or "f32": the storage type of a case's X."""
+    return "bf16" if str(c.X.dtype) == "torch.bfloat16" else "f32"
 
 
 def make_inputs(cases, seed=0):
@@ -141,8 +157,62 @@ def profile_traffic(kernel_key: str, source_file: str):
 
 
 # ----------------------------------------------------------------------------- clocks
-class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons while the GPU works."""
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML every `period_s` from a host
+    thread (reading only; nothing is set).  A timed region of a few tens of
+    milliseconds still collects tens of samples this way."""
+
+    def __init__(self, uuid: str, period_s: float = 0.002):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.period = period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self.thread = None
+        get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        self._reasons = get
+        self._bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                      pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+
+    def start(self):
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = int(self._reasons(self.h))
+                self.samples.append((time.time(), mhz, r))
+            except Exception:  # a failed read is skipped, not fatal
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "source": "nvml"}
+        reasons = sorted({REASON_NAMES[i] for (_, _, r) in inside for i, b in enumerate(self._bits) if r & b})
+        return {"sm_mhz": statistics.median(m for (_, m, _) in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "source": "nvml"}
+
+
+class SmiClockSampler:
+    """Fallback: nvidia-smi sampling of SM clock and throttle reasons while the GPU works."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
@@ -184,7 +254,7 @@ class ClockSampler:
     def summary(self, t0, t1):
         inside = [p for (t, p) in self.samples if t0 <= t <= t1] or [p for (_, p) in self.samples]
         if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0, "source": "smi"}
 
         def num(x):
             try:
@@ -193,10 +263,23 @@ class ClockSampler:
                 return None
         sm = [num(p[0]) for p in inside if num(p[0]) is not None]
         mx = [num(p[1]) for p in inside if num(p[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for p in inside for i in range(4) if p[3 + i].lower() == "active"})
+        reasons = sorted({REASON_NAMES[i] for p in inside for i in range(4) if p[3 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(inside)}
+                "reasons": reasons, "samples": len(inside), "source": "smi"}
+
+
+def clock_sampler(props):
+    """NVML sampler for this device (by UUID), else the nvidia-smi one."""
+    uuid = ""
+    try:
+        uuid = str(props.uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        pass
+    try:
+        return NvmlClockSampler(uuid)
+    except Exception:
+        return SmiClockSampler(uuid)
 
 
 # ----------------------------------------------------------------------------- distributed
@@ -284,22 +367,36 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_ours(args):
-    import torch
-    import ternary_weight_bit_b200 as tb
+def _timed_graph_replays(torch, graph, stream, min_s: float, max_reps: int = 100000):
+    """Replay `graph` on `stream` for at least min_s seconds (3 untimed replays first);
+    returns (milliseconds, replays), timed with CUDA events on that stream."""
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph.replay()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    one = max(e0.elapsed_time(e1), 1e-3)
+    reps = int(max(3, min(max_reps, math.ceil(min_s * 1e3 / one))))
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1), reps
 
-    world, rank, local = dist_setup(args.gpus)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
 
-    cases = workload_cases(args.workload)
+def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sampler, stream, sub_s=0.4, e2e=True):
+    """One forward workload on this rank: the timed steps (CUDA graphs, events on the
+    launching stream), then the dominant kernel alone, the activation kernel alone and
+    the end-to-end public call.  Returns the rank-local figures."""
+    cases = workload_cases(name)
     host = make_inputs(cases)
-    bf16_out = args.out_dtype == "bf16"
     if bf16_out and any(c.up is not None for c in host):
         raise SystemExit("--out-dtype bf16 applies to the plain forward workloads")
     out_dtype = torch.bfloat16 if bf16_out else torch.float32
@@ -315,6 +412,7 @@ def run_ours(args):
         del W
         base.append((packed, alpha))
     packed_bytes = sum(p.numel() for p, _ in base)
+
     def in_bytes(c):
         return c.X.numel() * c.X.element_size() * (2 if c.up is not None else 1)
 
@@ -347,10 +445,8 @@ def run_ours(args):
         for c, item in zip(host, rot[r]):
             forward(c, *item)
 
-    stream = torch.cuda.Stream(device=dev)
-    stream.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(stream):
-        for i in range(max(1, min(args.warmup, R))):
+        for i in range(max(1, min(warmup, R))):
             step(i % R)  # eager warm-up also primes the per-device attribute caches
     stream.synchronize()
     graphs = []
@@ -360,19 +456,10 @@ def run_ours(args):
             step(r)
         graphs.append(g)
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
+        for i in range(warmup):
             graphs[i % R].replay()
     stream.synchronize()
     assert tb.bitnet_get_last_device_status(stream) == 0
-
-    gpu_uuid = ""
-    try:
-        gpu_uuid = "GPU-" + str(props.uuid) if not str(props.uuid).startswith("GPU-") else str(props.uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_uuid)
-    sampler.start()
-    time.sleep(0.3)
 
     # ------------------------------------------------------------------ timed region
     if world > 1:
@@ -384,7 +471,7 @@ def run_ours(args):
     t_wall0 = time.time()
     e0.record(stream)
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
+        for i in range(steps):
             graphs[i % R].replay()
     e1.record(stream)
     e1.synchronize()
@@ -393,14 +480,14 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     elapsed = e0.elapsed_time(e1)
-    tokens_rank = args.steps * sum(c.M for c in host)
-    max_ms, tokens_all = aggregate(elapsed, tokens_rank, world, dev)
-    time.sleep(0.2)
-    sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler is not None else None
     status = tb.bitnet_get_last_device_status(stream)
+    tokens_rank = steps * sum(c.M for c in host)
+    kernels_per_step = sum(tb.bitnet_forward_kernel_count(c.M, c.N, c.K, c.fwht) for c in host)
 
     # ------------------------------------------------------------------ dominant kernel alone
+    peaks, peak_src = load_peaks()
+    decode_like = max(c.M for c in host) <= 16
     codes_scales = []
     for c, (X, p, a, out, ws, U) in zip(host, rot[0]):
         if U is None:
@@ -424,32 +511,18 @@ def run_ours(args):
     with torch.cuda.graph(gg, stream=stream):
         for r in range(R):
             gemm_pass(r)
-    reps = max(3, min(200, int(2000 / max(1, R * len(host)))))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            gg.replay()
-    k0 = torch.cuda.Event(enable_timing=True)
-    k1 = torch.cuda.Event(enable_timing=True)
-    k0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(reps):
-            gg.replay()
-    k1.record(stream)
-    k1.synchronize()
-    gemm_ms = k0.elapsed_time(k1)
+    gemm_ms, reps = _timed_graph_replays(torch, gg, stream, sub_s)
     launches = reps * R * len(host)
     gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32", out_bytes)[1] for c in host)
     gemm_ops = reps * R * sum(2.0 * c.M * c.N * c.K for c in host)
     weight_bytes = reps * R * sum(c.N * c.K / 4 for c in host)
     avg_launch_s = gemm_ms / 1e3 / launches
-    peaks, peak_src = load_peaks()
-    decode_like = max(c.M for c in host) <= 16
     if decode_like:
         achieved = gemm_bytes / launches / avg_launch_s / 1e9
         peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic(f"gemv_traffic_{args.workload}", "gemv.cu"),
+                "traffic": profile_traffic(f"gemv_traffic_{name}", "gemv.cu"),
                 "kernel": "gemv_kernel (register-streamed packed weights, mma.sync s8, in-CTA split-K)",
                 "peak_source": f"hbm_gbs of {peak_src} MEASURED_PEAKS.json (copy, burst)",
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
@@ -460,7 +533,7 @@ def run_ours(args):
         peak = 2.0 * bf16
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic(f"gemm_tc_traffic_{args.workload}", "gemm_sm100.cu"),
+                "traffic": profile_traffic(f"gemm_tc_traffic_{name}", "gemm_sm100.cu"),
                 "kernel": "gemm_tc_kernel (tcgen05 kind::i8, weights as TMEM A operand, TMEM accumulator)",
                 "peak_source": f"int8 dense = 2 x bf16_tflops of {peak_src} MEASURED_PEAKS.json (nominal ratio)",
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
@@ -480,18 +553,8 @@ def run_ours(args):
     with torch.cuda.graph(ga, stream=stream):
         for r in range(R):
             act_pass(r)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            ga.replay()
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(reps):
-            ga.replay()
-    a1.record(stream)
-    a1.synchronize()
-    act_s = a0.elapsed_time(a1) / 1e3 / (reps * R * len(host))
+    a_ms, a_reps = _timed_graph_replays(torch, ga, stream, sub_s)
+    act_s = a_ms / 1e3 / (a_reps * R * len(host))
     act_bytes = sum(in_bytes(c) + c.M * c.K + 4 * c.M for c in host) / len(host)
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     act = {"kernel": "act_quant (RMSNorm, FWHT when on, int8/int4 codes)", "bound": "hbm",
@@ -500,40 +563,90 @@ def run_ours(args):
            "frac": round(act_bytes / act_s / 1e9 / hbm, 4)}
 
     # ------------------------------------------------------------------ end to end through the public API
-    pinned_x = [c.X.pin_memory() for c in host]
-    pinned_u = [None if c.up is None else c.up.pin_memory() for c in host]
-    pinned_o = [torch.empty((c.M, c.N), dtype=out_dtype).pin_memory() for c in host]
-    e2e_steps = max(3, min(args.steps, 200))
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            for c, hx, hu, ho, (X, p, a, out, ws, U) in zip(host, pinned_x, pinned_u, pinned_o, rot[0]):
-                X.copy_(hx, non_blocking=True)
-                if U is not None:
-                    U.copy_(hu, non_blocking=True)
-                forward(c, X, p, a, out, ws, U)
-                ho.copy_(out, non_blocking=True)
-    stream.synchronize()
-    x0 = torch.cuda.Event(enable_timing=True)
-    x1 = torch.cuda.Event(enable_timing=True)
-    x0.record(stream)
-    with torch.cuda.stream(stream):
-        for i in range(e2e_steps):
+    e2e_res = None
+    if e2e:
+        pinned_x = [c.X.pin_memory() for c in host]
+        pinned_u = [None if c.up is None else c.up.pin_memory() for c in host]
+        pinned_o = [torch.empty((c.M, c.N), dtype=out_dtype).pin_memory() for c in host]
+
+        def e2e_step(i):
             for c, hx, hu, ho, (X, p, a, out, ws, U) in zip(host, pinned_x, pinned_u, pinned_o, rot[i % R]):
                 X.copy_(hx, non_blocking=True)
                 if U is not None:
                     U.copy_(hu, non_blocking=True)
                 forward(c, X, p, a, out, ws, U)
                 ho.copy_(out, non_blocking=True)
-    x1.record(stream)
-    x1.synchronize()
-    e2e_ms = x0.elapsed_time(x1)
-    e2e_max, e2e_tokens = aggregate(e2e_ms, e2e_steps * sum(c.M for c in host), world, dev)
-    h2d = sum(in_bytes(c) for c in host)
-    d2h = sum(out_bytes * c.M * c.N for c in host)
+
+        with torch.cuda.stream(stream):
+            for i in range(2):
+                e2e_step(i)
+        stream.synchronize()
+        e2e_steps = max(3, min(steps, 200))
+        x0 = torch.cuda.Event(enable_timing=True)
+        x1 = torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(e2e_steps):
+                e2e_step(i)
+        x1.record(stream)
+        x1.synchronize()
+        e2e_max, e2e_tokens = aggregate(x0.elapsed_time(x1), e2e_steps * sum(c.M for c in host), world, dev)
+        e2e_res = {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": sum(in_bytes(c) for c in host),
+                   "d2h_bytes_per_step": sum(out_bytes * c.M * c.N for c in host),
+                   "note": "eager calls of the public forward with pinned host inputs in and output out per step"}
+    for g in graphs:
+        del g
+    return {"cases": cases, "host": host, "R": R, "step_bytes": step_bytes, "elapsed_ms": elapsed,
+            "tokens_rank": tokens_rank, "clocks": clocks, "status": status, "roofline": roof,
+            "act_quant": act,
+            "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
+            "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1), "e2e": e2e_res,
+            "gpu_launches": steps * kernels_per_step}
+
+
+def run_ours(args):
+    import torch
+    import ternary_weight_bit_b200 as tb
+
+    world, rank, local = dist_setup(args.gpus)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    bf16_out = args.out_dtype == "bf16"
+    props = torch.cuda.get_device_properties(dev)
+    sampler = clock_sampler(props)
+    sampler.start()
+    time.sleep(0.05)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+
+    m = measure_forward(torch, tb, args.workload, dev, world, args.steps, args.warmup, bf16_out, sampler, stream)
+    max_ms, tokens_all = aggregate(m["elapsed_ms"], m["tokens_rank"], world, dev)
+    sub = None
+    if args.workload == DEFAULT_WORKLOAD and not args.no_decode_record:
+        # the decode configuration, same rules, in the same process: enough steps for
+        # about half a second of timed work
+        d_steps = max(args.steps, 2000)
+        d = measure_forward(torch, tb, "decode", dev, world, d_steps, args.warmup, bf16_out, sampler, stream,
+                            e2e=False)
+        d_ms, d_tok = aggregate(d["elapsed_ms"], d["tokens_rank"], world, dev)
+        sub = {"workload": workload_text("decode"), "name": "decode", "steps": d_steps, "warmup": args.warmup,
+               "value": round(d_tok / (d_ms / 1e3), 1), "unit": "tokens/s",
+               "ms_per_step": round(d_ms / d_steps, 6), "roofline": d["roofline"],
+               "act_quant": d["act_quant"], "gpu_launches": d["gpu_launches"],
+               "clocks": {k: d["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+               "device_status": d["status"]}
+    sampler.stop()
 
     result = None
     if rank == 0:
         value = tokens_all / (max_ms / 1e3)
+        R, step_bytes = m["R"], m["step_bytes"]
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6), "higher_is_better": True,
@@ -541,32 +654,34 @@ def run_ours(args):
             "config": {"workload": workload_text(args.workload), "name": args.workload,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} copies ({R * step_bytes / 2**20:.0f} MiB > 4x L2)"
-                       if R > 1 else "per-step working set larger than 4x L2",
+                       if R > 1 else f"per-step working set {step_bytes / 2**20:.0f} MiB, larger than 4x L2",
                        "cuda_graphs": True, "pdl": True, "out_dtype": args.out_dtype},
-            "roofline": roof,
-            "act_quant": act,
-            "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
-            "weight_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
-            "e2e": {"value": round(e2e_tokens / (e2e_max / 1e3), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "note": "eager calls of the public forward with pinned host inputs in and output out per step"},
-            "gpu_launches": args.steps * 2 * len(host),
-            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-            "device_status": status,
+            "roofline": m["roofline"],
+            "act_quant": m["act_quant"],
+            "gemm_tops": m["gemm_tops"],
+            "weight_gbs": m["weight_gbs"],
+            "e2e": m["e2e"],
+            "gpu_launches": m["gpu_launches"],
+            "clocks": {k: m["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples", "source")},
+            "device_status": m["status"],
         }
+        if sub is not None:
+            result["decode"] = sub
     # every rank has finished its GPU work; rank 0 now times the oracle on the host (N=1 only)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-        for g in graphs:
-            del g
-        graphs.clear()
         dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            v, desc, n, per_step = time_oracle(cases, budget_s=args.cpu_budget, bf16_out=bf16_out)
+            v, desc, n, per_step = time_oracle(m["cases"], budget_s=args.cpu_budget, bf16_out=bf16_out)
             result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                       "sample": desc}
+            if sub is not None:
+                v, desc, n, per_step = time_oracle(workload_cases("decode"), budget_s=max(3.0, args.cpu_budget / 3),
+                                                   bf16_out=bf16_out)
+                result["decode"]["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": 1,
+                                                    "kind": "oracle", "sample": desc}
         print(json.dumps(result), flush=True)
 
 
@@ -659,14 +774,9 @@ def run_kv(args):
         for i in range(args.warmup):
             graphs[i % R].replay()
     stream.synchronize()
-    gpu_uuid = ""
-    try:
-        gpu_uuid = "GPU-" + str(props.uuid) if not str(props.uuid).startswith("GPU-") else str(props.uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(gpu_uuid)
+    sampler = clock_sampler(props)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -686,7 +796,6 @@ def run_kv(args):
         dist.barrier()
     elapsed = e0.elapsed_time(e1)
     max_ms, tokens_all = aggregate(elapsed, args.steps * B * S, world, dev)
-    time.sleep(0.2)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
     status = tb.bitnet_get_last_device_status(stream)
@@ -760,7 +869,7 @@ def run_kv(args):
                                                                                for c, s in zip(pin_c, pin_s)),
                     "note": "eager bitnet_kv_quant calls with pinned host K, V in and codes, steps out per step"},
             "gpu_launches": 2 * args.steps,
-            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples", "source")},
             "device_status": status,
         }
     if world > 1:
@@ -847,8 +956,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode",
-                    help="decode (default) | prefill | wdown | wdown_swiglu | msweep_M<M> | kvcache")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help=f"{DEFAULT_WORKLOAD} (default) | decode | prefill | wdown | wdown_swiglu | msweep_M<M> | "
+                         "kvcache")
+    ap.add_argument("--no-decode-record", action="store_true",
+                    help="skip the decode sub-record of the default workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dtype", choices=["f32", "bf16"], default="f32",

@@ -14,8 +14,12 @@
  *   - Shapes: activations X [M][K], weights W [N][K] (the [out][in] layout of
  *     F.linear), output [M][N]; all row-major and densely packed.
  *   - Pointers: unless stated otherwise every pointer is a DEVICE pointer owned by
- *     the caller.  The library never allocates, frees or retains memory; it keeps
- *     only a per-device cache of kernel attributes and one 4-byte device status word.
+ *     the caller.  The library never allocates, frees or retains memory at run time.
+ *     Its own device memory is static, allocated when the library is loaded on a
+ *     device: one 4-byte status word and the fixed scratch array of
+ *     BITNET_NOALLOC_SCRATCH_BYTES (4 MiB) used only by
+ *     bitnet_hbitlinear_forward_noalloc.  On the host it keeps per-device caches of
+ *     kernel attributes and device addresses.
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call only enqueues work on that stream and returns without
  *     synchronising; results are ready when the stream reaches them.  The kernels
@@ -36,8 +40,10 @@
  *     that gives up on a bounded wait records BITNET_ERR_TIMEOUT in the device
  *     status word, which bitnet_get_last_device_status() reads.
  *   - Alignment: every device pointer must be 16-byte aligned (256-byte for
- *     workspaces).  K must be a multiple of 128 and at most 32768; with the FWHT on
- *     K must also be a power of two.  M >= 0 and N >= 1; M == 0 is a no-op.
+ *     workspaces).  K must be a multiple of 128 and at most 32768 (128 k is the step
+ *     of every kernel: one 128-byte row of codes and 32 bytes of packed weights per
+ *     row); with the FWHT on K must also be a power of two.  M >= 0 and N >= 1;
+ *     M == 0 is a no-op.
  *   - eps is the stabiliser of RMSNorm, of the activation scale and of the weight
  *     scale; the benchmarks use 1e-5.
  */
@@ -51,7 +57,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 6
+#define BITNET_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -103,6 +109,10 @@ typedef enum {
  * Deterministic: the same W always gives the same bytes and alpha.
  * ------------------------------------------------------------------------ */
 BITNET_API size_t bitnet_pack_workspace_bytes(int64_t N, int64_t K);
+/* One workspace size that serves every call on an M x N x K problem: the largest of
+ * bitnet_pack_workspace_bytes(N, K), bitnet_forward_workspace_bytes(M, K) and
+ * bitnet_gemm_workspace_bytes(M, N, K). */
+BITNET_API size_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K);
 BITNET_API bitnet_status_t bitnet_pack_ternary(const float *W, int64_t N, int64_t K, float eps,
                                     uint8_t *packed, float *alpha,
                                     void *ws, size_t ws_bytes, void *stream);
@@ -142,15 +152,25 @@ BITNET_API bitnet_status_t bitnet_act_quant(const void *X, bitnet_dtype_t xdt, i
  *   alpha    one fp32, device, read only.
  *   out      [M][N] fp32, device, written.
  *   acc_out  [M][N] int32, device, written when not NULL (for exactness checks).
+ *   ws       NULL, or device scratch of at least bitnet_gemm_workspace_bytes(M, N, K)
+ *            bytes (256-byte aligned; BITNET_ERR_WORKSPACE if smaller).  With a
+ *            workspace, a problem with few output tiles for the SMs may split K
+ *            over several CTAs per tile as bitnet_hbitlinear_forward does
+ *            (bitnet_forward_gemm_plan); the call then first zeroes the workspace's
+ *            counters (and, for more than two splits, `out`) with memsets on the
+ *            stream.  Without one, K is never split.  The result is bit-identical
+ *            either way.
  * M <= 16 runs the weight-streaming decode kernel (tensor-core mma.sync, split-K
- * over the warps of a CTA); larger M runs the persistent tcgen05 int8 tensor-core
- * GEMM with TMEM accumulators, whose token-tile size is chosen per shape (see
- * bitnet_gemm_token_tile below).
+ * over the warps of a CTA); larger M runs the persistent tcgen05
+ * int8 tensor-core GEMM with TMEM accumulators, whose token-tile size is chosen per
+ * shape (see bitnet_gemm_token_tile below).
  * ------------------------------------------------------------------------ */
+BITNET_API size_t bitnet_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 BITNET_API bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x,
                                     bitnet_act_mode_t mode, const uint8_t *packed,
                                     const float *alpha, int64_t M, int64_t N, int64_t K,
-                                    float *out, int32_t *acc_out, void *stream);
+                                    float *out, int32_t *acc_out, void *ws, size_t ws_bytes,
+                                    void *stream);
 
 /* --------------------------------------------------------------------------
  * bitnet_hbitlinear_forward -- the whole path: bitnet_act_quant into the
@@ -158,12 +178,18 @@ BITNET_API bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float 
  * programmatic dependent launch so its weight stream starts while the first runs).
  * Definition: bitnet_v2_engine.py page, HBitLinear.forward, Eq. 7.
  *   Arguments as in the two calls above; ws is device scratch of at least
- *   bitnet_forward_workspace_bytes(M, K) bytes holding the int8 codes and the
- *   per-token scales between the two kernels, and 4 KB of tile counters for a
- *   split-K GEMM (BITNET_ERR_WORKSPACE if smaller).  Its contents need no
- *   initialisation.
+ *   bitnet_forward_workspace_bytes(M, K) bytes holding the int8 codes [M][K] at
+ *   offset 0 and the per-token scales [M] at offset align256(M*K) between the two
+ *   kernels, and 4 KB of tile counters for a split-K GEMM (BITNET_ERR_WORKSPACE if
+ *   smaller).  Its contents need no initialisation; after the call the codes and
+ *   scales there are the ones the forward used.
+ * bitnet_forward_kernel_count: the number of kernels the forward launches for an
+ *   M x N x K problem with the FWHT on or off and with or without a gain (2: the
+ *   activation kernel and the decode kernel or the tcgen05 GEMM; 0 for M == 0; -1 for
+ *   sizes the forward rejects).  Host-only, no CUDA call.
  * ------------------------------------------------------------------------ */
 BITNET_API size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K);
+BITNET_API int bitnet_forward_kernel_count(int64_t M, int64_t N, int64_t K, int fwht, int has_gain);
 BITNET_API bitnet_status_t bitnet_hbitlinear_forward(const void *X, bitnet_dtype_t xdt, int64_t M,
                                           int64_t K, const float *gain, float eps, int fwht,
                                           bitnet_act_mode_t mode, const uint8_t *packed,

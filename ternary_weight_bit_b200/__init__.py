@@ -26,7 +26,8 @@ __all__ = [
     "bitnet_hbitlinear_forward", "bitnet_hbitlinear_forward_noalloc", "bitnet_forward_workspace_bytes", "bitnet_pack_workspace_bytes",
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
     "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_gemm_force_k_splits",
-    "bitnet_forward_gemm_plan",
+    "bitnet_forward_gemm_plan", "bitnet_workspace_bytes", "bitnet_gemm_workspace_bytes",
+    "bitnet_forward_kernel_count",
     "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu", "bitnet_kv_quant",
     "bitnet_ternary_gemm_ex", "bitnet_hbitlinear_forward_ex",
 ]
@@ -93,6 +94,21 @@ def bitnet_gemm_force_k_splits(k_splits: int) -> None:
 
 def bitnet_pack_workspace_bytes(N: int, K: int) -> int:
     return _native.load().bitnet_pack_workspace_bytes(N, K)
+
+
+def bitnet_workspace_bytes(M: int, N: int, K: int) -> int:
+    """One workspace size that serves pack, forward and GEMM on an M x N x K problem."""
+    return _native.load().bitnet_workspace_bytes(M, N, K)
+
+
+def bitnet_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return _native.load().bitnet_gemm_workspace_bytes(M, N, K)
+
+
+def bitnet_forward_kernel_count(M: int, N: int, K: int, fwht: bool = True, gain: bool = False) -> int:
+    """Kernels the forward launches for this problem (1 when the decode kernel runs the
+    activation step itself, else 2; 0 for M == 0; -1 for rejected sizes)."""
+    return _native.load().bitnet_forward_kernel_count(M, N, K, int(bool(fwht)), int(bool(gain)))
 
 
 def bitnet_forward_workspace_bytes(M: int, K: int) -> int:
@@ -214,8 +230,11 @@ def bitnet_kv_quant(kv: torch.Tensor, bits: int = 4, eps: float = 1e-5, dequant:
 
 
 def bitnet_ternary_gemm(codes: torch.Tensor, scale_x: torch.Tensor, mode, packed: torch.Tensor,
-                        alpha: torch.Tensor, N: int, out=None, acc_out=None, stream=None):
-    """acc = codes @ t^T (exact int32) and out = acc * (alpha * scale_x / Q).  Returns out fp32 [M, N]."""
+                        alpha: torch.Tensor, N: int, out=None, acc_out=None, ws=None, stream=None):
+    """acc = codes @ t^T (exact int32) and out = acc * (alpha * scale_x / Q).  Returns out fp32 [M, N].
+
+    ws (optional, uint8, >= bitnet_gemm_workspace_bytes) lets a problem with few output
+    tiles split K; without it K is never split.  The result is the same either way."""
     L = _native.load()
     _need(codes, "codes", torch.int8)
     M, K = codes.shape
@@ -226,9 +245,12 @@ def bitnet_ternary_gemm(codes: torch.Tensor, scale_x: torch.Tensor, mode, packed
     _need(out, "out", torch.float32, (M, N))
     if acc_out is not None:
         _need(acc_out, "acc_out", torch.int32, (M, N))
+    if ws is not None:
+        _need(ws, "ws", torch.uint8)
     _native.check("bitnet_ternary_gemm",
                   L.bitnet_ternary_gemm(_ptr(codes), _ptr(scale_x), mode_id(mode), _ptr(packed), _ptr(alpha), M, N,
-                                        K, _ptr(out), _ptr(acc_out), _stream(stream)))
+                                        K, _ptr(out), _ptr(acc_out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                        _stream(stream)))
     return out
 
 

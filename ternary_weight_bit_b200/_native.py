@@ -57,7 +57,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_pack_workspace_bytes": (SZ, [I64, I64]),
         "bitnet_pack_ternary": (I, [P, I64, I64, F, P, P, P, SZ, P]),
         "bitnet_act_quant": (I, [P, I, I64, I64, P, F, I, I, P, P, P]),
-        "bitnet_ternary_gemm": (I, [P, P, I, P, P, I64, I64, I64, P, P, P]),
+        "bitnet_ternary_gemm": (I, [P, P, I, P, P, I64, I64, I64, P, P, P, SZ, P]),
+        "bitnet_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
+        "bitnet_workspace_bytes": (SZ, [I64, I64, I64]),
+        "bitnet_forward_kernel_count": (I, [I64, I64, I64, I, I]),
         "bitnet_forward_workspace_bytes": (SZ, [I64, I64]),
         "bitnet_hbitlinear_forward": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P, SZ, P]),
         "bitnet_hbitlinear_forward_noalloc": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P]),

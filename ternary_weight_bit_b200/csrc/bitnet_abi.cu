@@ -144,21 +144,34 @@ bitnet_status_t validate_act(const void *X, int xdt, int64_t M, int64_t K, const
     return BITNET_OK;
 }
 
+// The standalone GEMM.  With a workspace (tile_cnt, kSplitCounters ints) an fp32
+// GEMM of few output tiles may split K as the forward does; the counters (and, for
+// more than two splits, the output) are zeroed by memsets on the stream first.
 cudaError_t run_gemm(const int8_t *codes, const float *scale_x, int mode, const uint8_t *packed,
                      const float *alpha, int64_t M, int64_t N, int64_t K, void *out, bool out_bf16,
-                     int32_t *acc_out, bool pdl, cudaStream_t s) {
+                     int32_t *acc_out, bool pdl, cudaStream_t s, int *tile_cnt = nullptr) {
     if (M <= kGemvMaxM)
         return launch_gemv(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s,
                            out_bf16);
-    return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s,
-                          GemmPlan{0, 1}, nullptr, out_bf16);
+    GemmPlan plan{0, 1};
+    if (tile_cnt && !out_bf16) {
+        plan = gemm_plan((int)M, (int)N, (int)K, sm_count(), kSplitCounters);
+        if (plan.splits > 1) {
+            cudaError_t e = cudaMemsetAsync(tile_cnt, 0, (size_t)kSplitCounters * sizeof(int), s);
+            if (e == cudaSuccess && plan.splits > 2) e = cudaMemsetAsync(out, 0, (size_t)M * (size_t)N * 4, s);
+            if (e != cudaSuccess) return e;
+            pdl = false;  // the kernel follows a memset, not a kernel
+        }
+    }
+    return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, acc_out, pdl, s, plan,
+                          plan.splits > 1 ? tile_cnt : nullptr, out_bf16);
 }
 
 }  // namespace
 
 // act_quant into (codes, scale_x), then the GEMV or the tcgen05 GEMM, the second
-// launched with programmatic dependent launch.  A GEMM whose output has few tiles
-// splits K: act_quant then also zeroes `out` and the tile counters for it.
+// launched with programmatic dependent launch.  A GEMM whose output has few tiles splits K:
+// act_quant then also zeroes `out` and the tile counters for it.
 cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain, float eps,
                             int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
                             int64_t N, void *out, int8_t *codes, float *scale_x, int *tile_cnt, cudaStream_t s,
@@ -187,6 +200,18 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
                            out_bf16);
     return launch_gemm_tc(codes, scale_x, mode, packed, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s, plan,
                           tile_cnt, out_bf16);
+}
+
+// Argument rules of every forward entry point (workspace excluded).
+bitnet_status_t validate_forward(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain,
+                                 int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
+                                 int64_t N, const void *out) {
+    if (N < 1 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
+    bitnet_status_t st = validate_act(X, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
+    if (st != BITNET_OK || M == 0) return st;
+    if (!packed || !alpha || !out || !aligned16(packed) || !aligned16(alpha) || !aligned16(out))
+        return BITNET_ERR_INVALID_ARG;
+    return BITNET_OK;
 }
 
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s) {
@@ -244,11 +269,13 @@ bitnet_status_t bitnet_act_quant(const void *X, bitnet_dtype_t xdt, int64_t M, i
 
 bitnet_status_t bitnet_ternary_gemm(const int8_t *codes, const float *scale_x, bitnet_act_mode_t mode,
                                     const uint8_t *packed, const float *alpha, int64_t M, int64_t N, int64_t K,
-                                    float *out, int32_t *acc_out, void *stream) {
+                                    float *out, int32_t *acc_out, void *ws, size_t ws_bytes, void *stream) {
     bitnet_status_t st = validate_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, acc_out);
     if (st != BITNET_OK || M == 0) return st;
+    if (ws && (ws_bytes < bitnet_gemm_workspace_bytes(M, N, K) || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return BITNET_ERR_WORKSPACE;
     return from_cuda(run_gemm(codes, scale_x, mode, packed, alpha, M, N, K, out, false, acc_out, true,
-                              static_cast<cudaStream_t>(stream)));
+                              static_cast<cudaStream_t>(stream), static_cast<int *>(ws)));
 }
 
 bitnet_status_t bitnet_ternary_gemm_ex(const int8_t *codes, const float *scale_x, bitnet_act_mode_t mode,
@@ -268,16 +295,29 @@ size_t bitnet_forward_workspace_bytes(int64_t M, int64_t K) {
            (size_t)kSplitCounters * sizeof(int);
 }
 
+size_t bitnet_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    (void)M;
+    (void)N;
+    (void)K;
+    return (size_t)kSplitCounters * sizeof(int);  // tile counters and ready flags of a split K
+}
+
+size_t bitnet_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    size_t need = bitnet_pack_workspace_bytes(N, K);
+    const size_t f = bitnet_forward_workspace_bytes(M, K), g = bitnet_gemm_workspace_bytes(M, N, K);
+    if (f > need) need = f;
+    if (g > need) need = g;
+    return need;
+}
+
+
 namespace {
 bitnet_status_t forward_ws(const void *X, const void *up, bitnet_dtype_t xdt, int64_t M, int64_t K,
                            const float *gain, float eps, int fwht, bitnet_act_mode_t mode, const uint8_t *packed,
                            const float *alpha, int64_t N, void *out, bool out_bf16, void *ws, size_t ws_bytes,
                            void *stream) {
-    if (N < 1 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
-    bitnet_status_t st = validate_act(X, xdt, M, K, gain, fwht, mode, nullptr, nullptr, false);
+    bitnet_status_t st = validate_forward(X, xdt, M, K, gain, fwht, mode, packed, alpha, N, out);
     if (st != BITNET_OK || M == 0) return st;
-    if (!packed || !alpha || !out || !aligned16(packed) || !aligned16(alpha) || !aligned16(out))
-        return BITNET_ERR_INVALID_ARG;
     if (!ws || ws_bytes < bitnet_forward_workspace_bytes(M, K) || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return BITNET_ERR_WORKSPACE;
     int8_t *codes = static_cast<int8_t *>(ws);
@@ -331,6 +371,13 @@ int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {
     if (M < 0 || N < 1 || N > kMaxRows || check_k(K, 0) != BITNET_OK) return -1;
     if (M <= kGemvMaxM) return 0;
     return gemm_pick_tile((int)M, (int)N, (int)K, sm_count());
+}
+
+int bitnet_forward_kernel_count(int64_t M, int64_t N, int64_t K, int fwht, int has_gain) {
+    (void)has_gain;
+    if (M < 0 || N < 1 || N > kMaxRows || M > kMaxRows || (fwht != 0 && fwht != 1)) return -1;
+    if (check_k(K, fwht) != BITNET_OK) return -1;
+    return M == 0 ? 0 : 2;  // act_quant, then the decode kernel or the tcgen05 GEMM
 }
 
 int bitnet_forward_gemm_plan(int64_t M, int64_t N, int64_t K, int *k_splits) {

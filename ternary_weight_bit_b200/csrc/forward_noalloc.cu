@@ -12,7 +12,13 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds it (kNoAllocScratchBytes) until the process exits.  Its host-side
 // name is only a stand-in for the device symbol; the kernels receive the device
-// address obtained from cudaGetSymbolAddress, looked up once per device.
+// address obtained from cudaGetSymbolAddress, looked up once per device and kept in
+// an atomic per-device cache (two host threads making their first call on a device at
+// once both look it up and store the same address).  cudaDeviceReset destroys the
+// module's device memory: after one, the cached address is stale, so a process that
+// resets a device must not call this entry point on it again.
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -28,27 +34,26 @@ constexpr size_t kNoAllocScratchBytes = BITNET_NOALLOC_SCRATCH_BYTES;
 // Shared by every call on a device; holds the last call's codes and scales.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-uint8_t *g_scratch_addr[kMaxDevices] = {};
+std::atomic<uint8_t *> g_scratch_addr[kMaxDevices];
 
 size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Device address of this device's scratch array (set up on first use per device).
+// Device address of this device's scratch array (set up on first use per device,
+// with that device current).
 cudaError_t scratch_address(uint8_t **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (!g_scratch_addr[dev]) {
-        uint8_t *p = nullptr;
+    uint8_t *p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         e = cudaGetSymbolAddress((void **)&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_release);
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -61,17 +66,9 @@ extern "C" bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
                                                               bitnet_act_mode_t mode, const uint8_t *packed,
                                                               const float *alpha, int64_t N, float *out,
                                                               void *stream) {
-    // Argument rules are those of bitnet_hbitlinear_forward.
-    if (xdt != BITNET_F32 && xdt != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
-    if (mode != BITNET_ACT_INT8_ABSMAX && mode != BITNET_ACT_INT4_ABSMEAN) return BITNET_ERR_INVALID_ARG;
-    if (fwht != 0 && fwht != 1) return BITNET_ERR_INVALID_ARG;
-    if (M < 0 || N < 1 || M > ((int64_t)1 << 30) || N > ((int64_t)1 << 30)) return BITNET_ERR_INVALID_ARG;
-    if (K <= 0 || K % 128 != 0 || K > 32768) return BITNET_ERR_UNSUPPORTED_SHAPE;
-    if (fwht && (K & (K - 1)) != 0) return BITNET_ERR_NOT_POW2;
-    if (M == 0) return BITNET_OK;
-    if (!X || !packed || !alpha || !out) return BITNET_ERR_INVALID_ARG;
-    if (!aligned16(X) || !aligned16(packed) || !aligned16(alpha) || !aligned16(out) || (gain && !aligned16(gain)))
-        return BITNET_ERR_INVALID_ARG;
+    // The argument rules of bitnet_hbitlinear_forward, from the same validator.
+    const bitnet_status_t st = validate_forward(X, xdt, M, K, gain, fwht, mode, packed, alpha, N, out);
+    if (st != BITNET_OK || M == 0) return st;
     // Codes [M][K], scales [M] (each 256-byte aligned) and the split-K tile counters
     // must fit the fixed array.
     const size_t codes_bytes = round256((size_t)M * (size_t)K);
@@ -84,8 +81,10 @@ extern "C" bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
     int8_t *codes = reinterpret_cast<int8_t *>(scratch);
     float *scale_x = reinterpret_cast<float *>(scratch + codes_bytes);
     int *tile_cnt = reinterpret_cast<int *>(scratch + codes_bytes + scales_bytes);
-    // Nothing in the array needs clearing beforehand: act_quant writes every code and
-    // scale the GEMM reads, and zeroes the counters when the GEMM splits K.
+    // Nothing in the array needs clearing beforehand: the forward's first kernel writes
+    // every code and scale that is read afterwards (the decode kernel that runs the
+    // activation step itself writes them for the record only), and act_quant zeroes
+    // the counters when the GEMM splits K.
     const cudaError_t e = forward_kernels(X, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, codes, scale_x,
                                           tile_cnt, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;

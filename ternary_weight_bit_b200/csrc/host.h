@@ -105,6 +105,12 @@ cudaError_t forward_kernels(const void *X, bitnet_dtype_t xdt, int64_t M, int64_
 cudaError_t launch_kv_quant(const void *kv, bool bf16, int64_t BH, int64_t S, int D, int bits, float eps,
                             int8_t *codes, float *step, float *deq, cudaStream_t s);
 
+// Argument rules shared by every forward entry point (the workspace is checked by
+// each entry point): BITNET_OK or the status the call returns.
+bitnet_status_t validate_forward(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K, const float *gain,
+                                 int fwht, bitnet_act_mode_t mode, const uint8_t *packed, const float *alpha,
+                                 int64_t N, const void *out);
+
 // Launch the timeout self-test kernel.
 cudaError_t launch_wait_selftest(uint32_t limit_us, cudaStream_t s);
 

@@ -2,6 +2,7 @@
 every function include/bitnet.h declares, and its argument validation rejects bad
 calls before any CUDA work is attempted."""
 import ctypes
+import re
 
 import pytest
 
@@ -27,7 +28,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 6
+    assert L.bitnet_abi_version() == 7
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
@@ -107,6 +108,39 @@ def test_out_dtype_validation(L):
     assert L.bitnet_ternary_gemm_ex(None, None, 0, None, None, 0, 256, 256, None, 1, None, s) == _native.OK  # M = 0
 
 
+# The boundary's calls with their parameter lists, as include/bitnet.h declares them.
+BOUNDARY = {
+    "bitnet_pack_ternary": ["const float *W", "int64_t N", "int64_t K", "float eps", "uint8_t *packed",
+                            "float *alpha", "void *ws", "size_t ws_bytes", "void *stream"],
+    "bitnet_act_quant": ["const void *X", "bitnet_dtype_t xdt", "int64_t M", "int64_t K", "const float *gain",
+                         "float eps", "int fwht", "bitnet_act_mode_t mode", "int8_t *codes", "float *scale_x",
+                         "void *stream"],
+    "bitnet_ternary_gemm": ["const int8_t *codes", "const float *scale_x", "bitnet_act_mode_t mode",
+                            "const uint8_t *packed", "const float *alpha", "int64_t M", "int64_t N", "int64_t K",
+                            "float *out", "int32_t *acc_out", "void *ws", "size_t ws_bytes", "void *stream"],
+    "bitnet_hbitlinear_forward": ["const void *X", "bitnet_dtype_t xdt", "int64_t M", "int64_t K",
+                                  "const float *gain", "float eps", "int fwht", "bitnet_act_mode_t mode",
+                                  "const uint8_t *packed", "const float *alpha", "int64_t N", "float *out",
+                                  "void *ws", "size_t ws_bytes", "void *stream"],
+    "bitnet_workspace_bytes": ["int64_t M", "int64_t N", "int64_t K"],
+    "bitnet_status_string": ["bitnet_status_t status"],
+    "bitnet_get_last_device_status": ["void *stream"],
+}
+
+
+def _declared_params(name):
+    src = open(_native.HEADER).read()
+    m = re.search(r"BITNET_API[^;]*?\b" + name + r"\s*\(([^)]*)\)\s*;", src, re.S)
+    assert m, f"{name} is not declared in bitnet.h"
+    return [" ".join(p.split()) for p in m.group(1).split(",")]
+
+
+def test_boundary_calls_have_their_listed_signatures(L):
+    for name, params in BOUNDARY.items():
+        assert _declared_params(name) == params, name
+        assert hasattr(L, name)
+
+
 def test_workspace_sizes(L):
     cnt = 4096  # split-K tile counters
     assert L.bitnet_forward_workspace_bytes(0, 256) == 0
@@ -114,6 +148,29 @@ def test_workspace_sizes(L):
     assert L.bitnet_forward_workspace_bytes(3, 2560) == 7680 + 256 + cnt
     assert L.bitnet_forward_workspace_bytes(100, 128) == 12800 + 512 + cnt
     assert L.bitnet_pack_workspace_bytes(6912, 2560) >= 8 * 1184
+    assert L.bitnet_gemm_workspace_bytes(64, 4096, 16384) == cnt
+    for M, N, K in ((1, 6912, 2560), (64, 4096, 16384), (8192, 4096, 4096)):
+        assert L.bitnet_workspace_bytes(M, N, K) == max(L.bitnet_pack_workspace_bytes(N, K),
+                                                        L.bitnet_forward_workspace_bytes(M, K),
+                                                        L.bitnet_gemm_workspace_bytes(M, N, K))
+
+
+def test_forward_kernel_count(L):
+    # the activation kernel, then the decode kernel or the tcgen05 GEMM; answered on the host
+    assert L.bitnet_forward_kernel_count(1, 6912, 2560, 0, 0) == 2
+    assert L.bitnet_forward_kernel_count(4096, 4096, 4096, 1, 1) == 2
+    assert L.bitnet_forward_kernel_count(0, 4096, 4096, 0, 0) == 0
+    assert L.bitnet_forward_kernel_count(4, 4096, 2560, 1, 0) == -1     # FWHT needs a power of two
+    assert L.bitnet_forward_kernel_count(4, 0, 4096, 0, 0) == -1
+
+
+def test_gemm_workspace_validation(L):
+    s = P(0)
+    # a workspace is optional; one that is given must be large enough and 256-byte aligned
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 64, 256, 256, FAKE, None, FAKE, 16, s) == \
+        _native.ERR_WORKSPACE
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 64, 256, 256, FAKE, None, P(4096 + 16), 1 << 20, s) == \
+        _native.ERR_WORKSPACE
 
 
 P = ctypes.c_void_p
@@ -133,18 +190,18 @@ def test_validation_rejects_bad_shapes(L):
     # bad enums
     assert L.bitnet_act_quant(FAKE, 7, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
     assert L.bitnet_act_quant(FAKE, 0, 4, 256, None, 1e-5, 0, 9, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
-    assert L.bitnet_ternary_gemm(FAKE, FAKE, 3, FAKE, FAKE, 4, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 3, FAKE, FAKE, 4, 16, 256, FAKE, None, None, 0, s) == _native.ERR_INVALID_ARG
     # negative sizes, N = 0
-    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, -1, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
-    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 0, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, -1, 16, 256, FAKE, None, None, 0, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 0, 256, FAKE, None, None, 0, s) == _native.ERR_INVALID_ARG
 
 
 def test_validation_rejects_bad_pointers(L):
     s = P(0)
     assert L.bitnet_act_quant(None, 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
     assert L.bitnet_act_quant(P(4100), 0, 4, 256, None, 1e-5, 0, 0, FAKE, FAKE, s) == _native.ERR_INVALID_ARG
-    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, None, FAKE, 4, 16, 256, FAKE, None, s) == _native.ERR_INVALID_ARG
-    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 16, 256, P(4104), None, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, None, FAKE, 4, 16, 256, FAKE, None, None, 0, s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm(FAKE, FAKE, 0, FAKE, FAKE, 4, 16, 256, P(4104), None, None, 0, s) == _native.ERR_INVALID_ARG
     assert L.bitnet_pack_ternary(FAKE, 16, 256, 1e-5, FAKE, FAKE, None, 0, s) == _native.ERR_WORKSPACE
     assert L.bitnet_pack_ternary(FAKE, 16, 256, 1e-5, FAKE, P(4108), FAKE, 1 << 20, s) == _native.ERR_INVALID_ARG
     # forward workspace too small, or misaligned
@@ -159,7 +216,7 @@ def test_validation_rejects_bad_pointers(L):
 def test_empty_batch_is_a_noop(L):
     s = P(0)
     assert L.bitnet_act_quant(None, 0, 0, 256, None, 1e-5, 1, 0, None, None, s) == _native.OK
-    assert L.bitnet_ternary_gemm(None, None, 0, None, None, 0, 16, 256, None, None, s) == _native.OK
+    assert L.bitnet_ternary_gemm(None, None, 0, None, None, 0, 16, 256, None, None, None, 0, s) == _native.OK
     assert L.bitnet_hbitlinear_forward(None, 0, 0, 256, None, 1e-5, 1, 0, FAKE, FAKE, 16, FAKE, None, 0,
                                        s) == _native.OK
 

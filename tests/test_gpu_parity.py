@@ -194,6 +194,32 @@ def test_gemm_forced_token_tiles(tile):
         tb.bitnet_gemm_force_token_tile(0)
 
 
+DECODE_SHAPES = [
+    (1, 11008, 4096),    # many weight rows
+    (3, 4096, 16384),    # a long row: many chunks per warp
+    (5, 700, 2944),      # K % 256 == 128: a half chunk at the end; ragged rows
+    (16, 2000, 384),     # two token groups of 8
+    (9, 37, 128),        # fewer weight rows than one CTA's, the last block ragged
+    (2, 6912, 2560), (8, 2560, 6912),
+]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_gemv_decode_kernel_shapes(M, N, K):
+    # the decode kernel on long and short rows, many weight rows, a half chunk at the
+    # end of K and ragged tails; exact accumulators, fp32 and bf16 outputs
+    mode = ("int8", "int4")[M % 2]
+    q, packed, scale, alpha = _gemm_case(M, N, K, mode, seed=M * 7 + N + K)
+    acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    out = tb.bitnet_ternary_gemm(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, acc_out=acc)
+    outh = tb.bitnet_ternary_gemm_ex(dev(q), dev(scale), mode, dev(packed), dev(alpha), N, out_dtype=torch.bfloat16)
+    acc_ref = ref.gemm_packed(q, packed, N)
+    np.testing.assert_array_equal(host(acc), acc_ref, err_msg=f"{M}x{N}x{K}")
+    out_ref = ref.dequant(acc_ref, scale, alpha[0], MODES[mode])
+    np.testing.assert_array_equal(host(out), out_ref)
+    np.testing.assert_array_equal(parity.bf16_bits(outh), ref.round_bf16(out_ref))
+
+
 def test_gemm_extreme_codes():
     # every code at the int8 extremes, every weight +1/-1: |acc| = 128 K is the largest possible
     for M, N, K in [(4, 64, 16384), (32, 256, 16384)]:
@@ -293,11 +319,26 @@ def test_forward_bf16_output_prefill_sampled():
 
 
 # ----------------------------------------------------------------------------- whole forward
+def _align256(v):
+    return (v + 255) // 256 * 256
+
+
+def ws_codes_scales(ws, M, K):
+    """The codes [M, K] and per-token scales [M] a forward left in its workspace."""
+    codes = ws[:M * K].view(torch.int8).view(M, K)
+    off = _align256(M * K)
+    scales = ws[off:off + 4 * M].view(torch.float32)
+    return codes, scales
+
+
 def _forward_case(case, sample_rows=None):
     Xd = case.X.to(DEV)
     W = case.W.to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(W, eps=case.eps)
-    out = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, case.N, eps=case.eps, fwht=case.fwht, mode=case.mode)
+    ws = torch.empty((tb.bitnet_forward_workspace_bytes(case.M, case.K),), dtype=torch.uint8, device=DEV)
+    out = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, case.N, eps=case.eps, fwht=case.fwht, mode=case.mode,
+                                       ws=ws)
+    fcodes, fscale = ws_codes_scales(ws, case.M, case.K)  # what the forward used
     codes, gscale = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=case.fwht, mode=case.mode)
     torch.cuda.synchronize()
     rows = np.arange(case.M) if sample_rows is None else sample_rows
@@ -308,11 +349,15 @@ def _forward_case(case, sample_rows=None):
     mode = MODES[case.mode]
     r = ref.hbitlinear_forward(X32, p_ref, a_ref, case.N, eps=case.eps, fwht_on=case.fwht, mode=mode)
     sh = ref.shadow(X32, None, case.eps, case.fwht, mode)
-    gcodes = host(codes)[rows]
-    parity.check_codes(gcodes, r.codes, sh, case.name)
     gout = host(out)[rows]
-    gs = host(gscale)[rows]
-    parity.check_scale_bound(gs, r.scale_x, case.K, mode, case.name)
+    # the standalone activation step and the forward's own codes and scales (the decode
+    # kernel may quantise inside itself), each against the oracle
+    for label, cc, ss in (("act_quant", codes, gscale), ("forward", fcodes, fscale)):
+        gcodes = host(cc)[rows]
+        gs = host(ss)[rows]
+        parity.check_codes(gcodes, r.codes, sh, f"{case.name} {label}")
+        parity.check_scale_bound(gs, r.scale_x, case.K, mode, f"{case.name} {label}")
+    gcodes, gs = host(fcodes)[rows], host(fscale)[rows]
     # same codes and scales -> identical output (exact accumulators, same IEEE steps)
     out_same = ref.dequant(ref.gemm_packed(gcodes, p_ref, case.N), gs, a_ref, mode)
     parity.check_out_same_codes(gout, out_same, case.name)
@@ -353,6 +398,11 @@ def _split_k_case(M, K, N, mode, fwht, seed):
     codes, scale = tb.bitnet_act_quant(Xd, eps=case.eps, fwht=fwht, mode=mode)
     out_unsplit = tb.bitnet_ternary_gemm(codes, scale, mode, packed, alpha, N)
     assert torch.equal(out, out_unsplit)
+    # the standalone GEMM given a workspace splits K the same way, to the same result
+    gws = torch.empty((tb.bitnet_gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device=DEV)
+    out_split = tb.bitnet_ternary_gemm(codes, scale, mode, packed, alpha, N, ws=gws)
+    out_split2 = tb.bitnet_ternary_gemm(codes, scale, mode, packed, alpha, N, ws=gws)  # counters left clean
+    assert torch.equal(out_split, out_unsplit) and torch.equal(out_split2, out_unsplit)
     assert tb.bitnet_get_last_device_status() == 0
 
 
@@ -406,7 +456,9 @@ def _swiglu_case(M, K, N, mode, fwht, xdt, seed, sample_rows=None):
         gate, up = gate.to(torch.bfloat16), up.to(torch.bfloat16)
     gd, ud = gate.to(DEV), up.to(DEV)
     packed, alpha = tb.bitnet_pack_ternary(W.to(DEV))
-    out = tb.bitnet_hbitlinear_forward_swiglu(gd, ud, packed, alpha, N, fwht=fwht, mode=mode)
+    ws = torch.empty((tb.bitnet_forward_workspace_bytes(M, K),), dtype=torch.uint8, device=DEV)
+    out = tb.bitnet_hbitlinear_forward_swiglu(gd, ud, packed, alpha, N, fwht=fwht, mode=mode, ws=ws)
+    fcodes, fscale = ws_codes_scales(ws, M, K)  # what the forward used
     codes, gscale = tb.bitnet_act_quant_swiglu(gd, ud, fwht=fwht, mode=mode)
     torch.cuda.synchronize()
     rows = np.arange(M) if sample_rows is None else sample_rows
@@ -415,8 +467,10 @@ def _swiglu_case(M, K, N, mode, fwht, xdt, seed, sample_rows=None):
     m = MODES[mode]
     r = ref.hbitlinear_forward(ref.swiglu(g32, u32), p_ref, a_ref, N, fwht_on=fwht, mode=m)
     sh = ref.shadow_swiglu(g32, u32, eps=1e-5, fwht_on=fwht, mode=m)
-    gcodes, gs, gout = host(codes)[rows], host(gscale)[rows], host(out)[rows]
     label = f"swiglu M={M} K={K} N={N} {mode} fwht={fwht} {xdt}"
+    parity.check_codes(host(codes)[rows], r.codes, sh, label + " act_quant")
+    parity.check_scale_bound(host(gscale)[rows], r.scale_x, K, m, label + " act_quant")
+    gcodes, gs, gout = host(fcodes)[rows], host(fscale)[rows], host(out)[rows]
     parity.check_codes(gcodes, r.codes, sh, label)
     parity.check_scale_bound(gs, r.scale_x, K, m, label)
     parity.check_out_same_codes(gout, ref.dequant(ref.gemm_packed(gcodes, p_ref, N), gs, a_ref, m), label)
@@ -549,7 +603,8 @@ def test_forward_chain_reads_the_previous_layers_output(M, fwht, mode):
         xin = host(xs[i]).astype(np.float32)
         p_ref, a_ref, _ = ref.pack_weights(W.numpy(), eps=1e-5)
         r = ref.hbitlinear_forward(xin, p_ref, a_ref, K, eps=1e-5, fwht_on=fwht, mode=MODES[mode])
-        codes, gs = tb.bitnet_act_quant(xs[i], eps=1e-5, fwht=fwht, mode=mode)
+        # the codes and scales this layer's forward used, left in its workspace
+        codes, gs = ws_codes_scales(layers[i].workspace(M, xs[i].device), M, K)
         gcodes = host(codes)
         sh = ref.shadow(xin, None, 1e-5, fwht, MODES[mode])
         label = f"chain layer {i} M={M}"
