@@ -227,14 +227,154 @@ __device__ __forceinline__ void zero_fill(const ZeroFill &z, int64_t token) {
         for (int i = threadIdx.x; i < z.cnt_n; i += blockDim.x) z.cnt[i] = 0;
 }
 
+// Per-token scalars shared through shared memory after a token's reduction.
+struct FwhtScalars {
+    float s_eff, stat;
+};
+
+// The FWHT and quantiser for one token whose phase-0 values are in v (thread tid owns
+// elements [tid*E, tid*E + E)); ss is this thread's partial sum of x^2.  Gain, log2 K
+// butterfly stages in phases of ELOG bits with shared-memory transposes between them,
+// then ONE block reduction of (sum x^2, max|z| or sum|z|) over the unscaled transform z:
+// RMSNorm's factor r and the 2^(-m/2) of the m stages are one scalar rho that commutes
+// with the transform, so y = rho z, gamma = rho max|z| (exact: rounding is monotone) or
+// beta = rho sum|z| / K, and the code is rne(z * (rho s)) -- the same values as scaling
+// first, up to the rounding of one product.  `hook` runs once every thread has read its
+// phase-0 values and passed the first transpose (the streaming kernel refills its input
+// buffer there).  Barriers: the first transpose needs none before its writes -- every
+// thread's previous reads of sm, red and sc were followed by this call's or the previous
+// call's reduction barriers.
+template <int LOGK, class Hook>
+__device__ __forceinline__ void fwht_quant_token(float (&v)[FwhtShape<LOGK>::E], float ss, int64_t token,
+                                                 const float *__restrict__ gain, float eps, int mode,
+                                                 int8_t *__restrict__ codes, float *__restrict__ scale_x, float *sm,
+                                                 float2 *red, FwhtScalars *sc, Hook hook) {
+    using S = FwhtShape<LOGK>;
+    constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
+    constexpr int W = T / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = token * K;
+
+    if (gain != nullptr) {
+#pragma unroll
+        for (int r = 0; r < E; ++r) v[r] = __fmul_rn(v[r], __ldg(gain + tid * E + r));
+    }
+
+    // Butterflies over all LOGK bits, in increasing bit order.
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        if (p > 0) {
+            if (p > 1) __syncthreads();  // every thread has read the previous phase's layout
+            float *wb = sm + pad(tid_part<LOGK, ELOG>(p - 1, tid));
+#pragma unroll
+            for (int r = 0; r < E; ++r) wb[pad(reg_part<LOGK, ELOG>(p - 1, r))] = v[r];
+            __syncthreads();
+            if (p == 1) hook();
+            const float *rb = sm + pad(tid_part<LOGK, ELOG>(p, tid));
+#pragma unroll
+            for (int r = 0; r < E; ++r) v[r] = rb[pad(reg_part<LOGK, ELOG>(p, r))];
+        } else if (P == 1) {
+            hook();
+        }
+        const int lo = p * ELOG;
+        const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
+        const int pass = ELOG - nb;
+#pragma unroll
+        for (int b = 0; b < ELOG; ++b) {
+            if (b >= pass) {
+                const int h = 1 << b;
+#pragma unroll
+                for (int r = 0; r < E; ++r) {
+                    if ((r & h) == 0) {
+                        const float a = v[r], c = v[r | h];
+                        v[r] = __fadd_rn(a, c);
+                        v[r | h] = __fsub_rn(a, c);
+                    }
+                }
+            }
+        }
+    }
+
+    // one reduction: (sum x^2, max|z| or sum|z|)
+    const bool mean = mode != BITNET_ACT_INT8_ABSMAX;
+    float st = 0.0f;
+    if (mean) {
+#pragma unroll
+        for (int r = 0; r < E; ++r) st += fabsf(v[r]);
+    } else {
+#pragma unroll
+        for (int r = 0; r < E; ++r) st = fmaxf(st, fabsf(v[r]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float x = __shfl_xor_sync(0xffffffffu, st, o);
+        st = mean ? st + x : fmaxf(st, x);
+    }
+    if constexpr (W > 1) {
+        if (lane == 0) red[warp] = make_float2(ss, st);
+        __syncthreads();
+        if (warp == 0) {
+            float2 q = lane < W ? red[lane] : make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                q.x += __shfl_xor_sync(0xffffffffu, q.x, o);
+                const float x = __shfl_xor_sync(0xffffffffu, q.y, o);
+                q.y = mean ? q.y + x : fmaxf(q.y, x);
+            }
+            ss = q.x;
+            st = q.y;
+        }
+    }
+    if (tid == 0) {
+        const float p2 = __int_as_float((127 - LOGK / 2) << 23);  // 2^(-floor(LOGK/2)), exact
+        const float hs = (LOGK & 1) ? __fmul_rn(0.70710678118654752f, p2) : p2;
+        const float rho = __fmul_rn(rms_factor(ss, K, eps), hs);
+        const float rs = __fmul_rn(rho, st);
+        const float stat = mean ? __fdiv_rn(rs, (float)K) : rs;
+        const QuantParams qp = quant_params(stat, eps, mode);
+        sc->s_eff = __fmul_rn(rho, qp.s);
+        sc->stat = stat;
+        scale_x[token] = stat;
+    }
+    __syncthreads();
+    const float s_eff = sc->s_eff;
+    const float lo = mean ? -8.0f : -128.0f, hi = mean ? 7.0f : 127.0f;
+    // int8: |z s_eff| <= 127 (1 + 4u) < 127.5, so the clip can never act.
+
+    // Store the codes in the last phase's layout.
+    constexpr int LASTLO = (P - 1) * ELOG;
+    constexpr int LASTNB = (LOGK - LASTLO) < ELOG ? (LOGK - LASTLO) : ELOG;
+    constexpr int LASTPASS = ELOG - LASTNB;
+    int8_t *out = codes + row + tid_part<LOGK, ELOG>(P - 1, tid);
+    if constexpr (LASTPASS >= 2) {
+#pragma unroll
+        for (int r = 0; r < E; r += 4) {
+            uint32_t f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = quant_bits(v[r + e], s_eff, lo, hi, mean);
+            *reinterpret_cast<uint32_t *>(out + reg_part<LOGK, ELOG>(P - 1, r)) = pack4_perm(f[0], f[1], f[2], f[3]);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < E; ++r)
+            out[reg_part<LOGK, ELOG>(P - 1, r)] = (int8_t)(quant_bits(v[r], s_eff, lo, hi, mean) & 0xFFu);
+    }
+}
+
+struct NoHook {
+    __device__ __forceinline__ void operator()() const {}
+};
+
 template <int LOGK, class Src>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::T)
 act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mode,
                       int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
     using S = FwhtShape<LOGK>;
-    constexpr int K = S::K, ELOG = S::ELOG, E = S::E, T = S::T, P = S::PHASES;
+    constexpr int K = S::K, E = S::E;
     extern __shared__ __align__(16) float sm[];  // K + K/32 floats (padded)
-    __shared__ float red[32];
+    __shared__ float2 red[32];
+    __shared__ FwhtScalars sc;
 
     // Let the GEMM launch now and start streaming its weights; then wait for X, which
     // may come from the previous kernel.  The GEMM waits for this kernel before it
@@ -259,91 +399,116 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
     float ss = 0.0f;
 #pragma unroll
     for (int r = 0; r < E; ++r) ss = fmaf(v[r], v[r], ss);
-    ss = block_sum<T>(ss, red);
-    const float rn = rms_factor(ss, K, eps);
+    fwht_quant_token<LOGK>(v, ss, blockIdx.x, gain, eps, mode, codes, scale_x, sm, red, &sc, NoHook{});
+}
 
-    if (gain != nullptr) {
-#pragma unroll
-        for (int r = 0; r < E; ++r) v[r] = __fmul_rn(v[r], __ldg(gain + tid * E + r));
-    }
+// ------------------------------------------------------------------ streaming FWHT kernel
+// For many tokens: a persistent grid whose CTAs loop over tokens (t = blockIdx.x,
+// + gridDim.x, ...).  Each token row is brought into shared memory by TMA tensor copies
+// (X viewed as [M][K/32][32], boxes of up to 256 rows of 32 elements, 128-byte (fp32)
+// or 64-byte (bf16) swizzled).  The copy of the CTA's next token is issued as soon as
+// every thread has read the current one (after the first transpose), so its HBM latency
+// overlaps the rest of the transform; one buffer per CTA keeps several CTAs resident
+// per SM.  The swizzle lets thread tid read its 32 contiguous elements (row tid of the
+// buffer) with 16-byte loads free of bank conflicts.  The transform is fwht_quant_token.
+template <int LOGK, bool BF16>
+struct StreamShape {
+    using S = FwhtShape<LOGK>;
+    static constexpr int K = S::K;
+    static constexpr int ROWS = K / 32;                         // 32-element rows per token
+    static constexpr int BOX = ROWS < 256 ? ROWS : 256;        // rows per TMA box
+    static constexpr int NBOX = ROWS / BOX;
+    static constexpr int XBYTES = K * (BF16 ? 2 : 4);          // one token row
+    static constexpr int TBYTES = (K + K / 32) * 4;            // transpose buffer
+    static constexpr int SMEM = XBYTES + TBYTES + 1024;        // + 1024-byte alignment
+};
 
-    // Butterflies over all LOGK bits, in increasing bit order.
+template <int LOGK, bool BF16>
+__global__ void __launch_bounds__(FwhtShape<LOGK>::T)
+act_quant_fwht_stream_kernel(const __grid_constant__ CUtensorMap tmx, const float *__restrict__ gain, float eps,
+                             int mode, int64_t M, int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf,
+                             int *status, const void *X) {
+    using S = FwhtShape<LOGK>;
+    using SS = StreamShape<LOGK, BF16>;
+    constexpr int E = S::E;
+    static_assert(E == 32, "one 32-element row per thread");
+    extern __shared__ uint8_t smraw[];
+    uint8_t *xbuf = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    float *sm = reinterpret_cast<float *>(xbuf + SS::XBYTES);  // transpose buffer
+    __shared__ float2 red[32];
+    __shared__ FwhtScalars sc;
+    __shared__ __align__(8) uint64_t full;
+    const int tid = threadIdx.x;
+
+    auto issue = [&](int64_t token) {  // thread 0: the whole row of `token` into the buffer
+        const uint32_t bar = smem_u32(&full);
+        asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                     "r"((uint32_t)SS::XBYTES)
+                     : "memory");
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
-        if (p > 0) {
-            __syncthreads();
-            float *wb = sm + pad(tid_part<LOGK, ELOG>(p - 1, tid));
-#pragma unroll
-            for (int r = 0; r < E; ++r) wb[pad(reg_part<LOGK, ELOG>(p - 1, r))] = v[r];
-            __syncthreads();
-            const float *rb = sm + pad(tid_part<LOGK, ELOG>(p, tid));
-#pragma unroll
-            for (int r = 0; r < E; ++r) v[r] = rb[pad(reg_part<LOGK, ELOG>(p, r))];
+        for (int j = 0; j < SS::NBOX; ++j)
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+                "[%2];" ::"r"(smem_u32(xbuf + j * SS::BOX * (BF16 ? 64 : 128))),
+                "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(bar), "r"(0), "r"(j * SS::BOX), "r"((int)token)
+                : "memory");
+    };
+    if (tid == 0) {
+        mbar_init(&full, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmx);
+        // X may come from the previous kernel: before the dependency wait only warm L2
+        for (int i = 0; i < 2; ++i) {
+            const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
+            if (t < M) bulk_prefetch_l2(reinterpret_cast<const uint8_t *>(X) + t * SS::XBYTES, SS::XBYTES);
         }
-        const int lo = p * ELOG;
-        const int nb = (LOGK - lo) < ELOG ? (LOGK - lo) : ELOG;
-        const int pass = ELOG - nb;
+    }
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();
+    __syncthreads();  // the barrier is initialised
+    if (tid == 0) issue(blockIdx.x);
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < M; t += gridDim.x, ++it) {
+        zero_fill(zf, t);  // a following split-K GEMM's output row (and, for token 0, its counters)
+        // bounded; on a timeout (recorded in the status word) the loop runs on, so that
+        // every thread still meets every barrier
+        mbar_wait(&full, (uint32_t)it & 1u, status);
+        // row tid of the buffer: 16-byte units swizzled by the row's position in its 1 KB block
+        float v[E];
+        if constexpr (BF16) {
 #pragma unroll
-        for (int b = 0; b < ELOG; ++b) {
-            if (b >= pass) {
-                const int h = 1 << b;
+            for (int u = 0; u < 4; ++u) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(xbuf + tid * 64 + ((u ^ ((tid >> 1) & 3)) << 4));
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int r = 0; r < E; ++r) {
-                    if ((r & h) == 0) {
-                        const float a = v[r], c = v[r | h];
-                        v[r] = __fadd_rn(a, c);
-                        v[r | h] = __fsub_rn(a, c);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    v[8 * u + 2 * i] = __uint_as_float(ww[i] << 16);
+                    v[8 * u + 2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
                 }
             }
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 w = *reinterpret_cast<const float4 *>(xbuf + tid * 128 + ((u ^ (tid & 7)) << 4));
+                v[4 * u] = w.x;
+                v[4 * u + 1] = w.y;
+                v[4 * u + 2] = w.z;
+                v[4 * u + 3] = w.w;
+            }
         }
+        float ss = 0.0f;
+#pragma unroll
+        for (int r = 0; r < E; ++r) ss = fmaf(v[r], v[r], ss);
+        const int64_t next = t + gridDim.x;
+        fwht_quant_token<LOGK>(v, ss, t, gain, eps, mode, codes, scale_x, sm, red, &sc, [&]() {
+            // every thread has read the buffer (the first transpose's barrier): refill it
+            if (tid == 0 && next < M) {
+                fence_proxy_async_smem();  // the reads are ordered before the copy's writes
+                issue(next);
+            }
+        });
     }
-
-    // y = z * (r * 2^(-LOGK/2))
-    const float p2 = __int_as_float((127 - LOGK / 2) << 23);  // 2^(-floor(LOGK/2)), exact
-    const float hs = (LOGK & 1) ? __fmul_rn(0.70710678118654752f, p2) : p2;
-    const float rho = __fmul_rn(rn, hs);
-    float stat;
-    if (mode == BITNET_ACT_INT8_ABSMAX) {
-        float mx = 0.0f;
-#pragma unroll
-        for (int r = 0; r < E; ++r) {
-            v[r] = __fmul_rn(v[r], rho);
-            mx = fmaxf(mx, fabsf(v[r]));
-        }
-        stat = block_max<T>(mx, red);
-    } else {
-        float sa = 0.0f;
-#pragma unroll
-        for (int r = 0; r < E; ++r) {
-            v[r] = __fmul_rn(v[r], rho);
-            sa += fabsf(v[r]);
-        }
-        stat = __fdiv_rn(block_sum<T>(sa, red), (float)K);
-    }
-    const QuantParams q = quant_params(stat, eps, mode);
-    // int8: |y| <= gamma makes |y*s| < 127.5, so the clip can never act.
-    const bool clip = mode != BITNET_ACT_INT8_ABSMAX;
-
-    // Store the codes in the last phase's layout.
-    constexpr int LASTLO = (P - 1) * ELOG;
-    constexpr int LASTNB = (LOGK - LASTLO) < ELOG ? (LOGK - LASTLO) : ELOG;
-    constexpr int LASTPASS = ELOG - LASTNB;
-    int8_t *out = codes + row + tid_part<LOGK, ELOG>(P - 1, tid);
-    if constexpr (LASTPASS >= 2) {
-#pragma unroll
-        for (int r = 0; r < E; r += 4) {
-            uint32_t f[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) f[e] = quant_bits(v[r + e], q.s, q.lo, q.hi, clip);
-            *reinterpret_cast<uint32_t *>(out + reg_part<LOGK, ELOG>(P - 1, r)) = pack4_perm(f[0], f[1], f[2], f[3]);
-        }
-    } else {
-#pragma unroll
-        for (int r = 0; r < E; ++r)
-            out[reg_part<LOGK, ELOG>(P - 1, r)] = (int8_t)(quant_bits(v[r], q.s, q.lo, q.hi, clip) & 0xFFu);
-    }
-    if (tid == 0) scale_x[blockIdx.x] = stat;
+    // every copy issued above was waited for in the loop before the CTA exits
 }
 
 // ------------------------------------------------------------------ plain kernel (no FWHT)
@@ -537,6 +702,36 @@ cudaError_t launch_fwht(const Src &src, int64_t M, const float *gain, float eps,
     return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, src, gain, eps, mode, codes, scale_x, zf);
 }
 
+// The streaming kernel for K = 2^LOGK, 11 <= LOGK <= 14 (T >= 64 threads, so that the
+// statistic's block reduction has barriers; two rows and the transpose buffer fit in
+// shared memory): a persistent grid of as many CTAs as the SMs hold.
+template <int LOGK, bool BF16>
+cudaError_t launch_fwht_stream(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
+                               float *scale_x, const ZeroFill &zf, cudaStream_t s) {
+    using S = FwhtShape<LOGK>;
+    using SS = StreamShape<LOGK, BF16>;
+    CUtensorMap tm;
+    if (!make_tmap_rows_3d(&tm, X, BF16, (uint64_t)S::K, (uint64_t)M, (uint32_t)SS::BOX))
+        return cudaErrorInvalidValue;
+    auto kern = act_quant_fwht_stream_kernel<LOGK, BF16>;
+    static int bps[kMaxDevices] = {};  // resident CTAs per SM
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int per_sm = dev < kMaxDevices ? bps[dev] : 0;
+    if (per_sm == 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SS::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, S::T, SS::SMEM);
+        if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+        if (dev < kMaxDevices) bps[dev] = per_sm;
+    }
+    const int64_t slots = (int64_t)per_sm * sm_count();
+    const int grid = (int)(M < slots ? M : slots);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(S::T), (size_t)SS::SMEM, s, tm, gain, eps, mode, M, codes,
+                      scale_x, zf, device_status_ptr(), X);
+}
+
 template <int NV8, class Src>
 cudaError_t launch_plain(const Src &src, int64_t M, int K, int T, const float *gain, float eps, int mode,
                          int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
@@ -544,10 +739,34 @@ cudaError_t launch_plain(const Src &src, int64_t M, int K, int T, const float *g
                       codes, scale_x, zf);
 }
 
+// Many tokens of a plain input with 2^11 <= K <= 2^14: the streaming FWHT kernel.
+template <class Src>
+cudaError_t dispatch_stream(const Src &, int64_t, int, const float *, float, int, int8_t *, float *, const ZeroFill &,
+                            cudaStream_t, bool &used) {
+    used = false;
+    return cudaSuccess;
+}
+template <bool BF16>
+cudaError_t dispatch_stream(const XSrc<BF16> &src, int64_t M, int K, const float *gain, float eps, int mode,
+                            int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s, bool &used) {
+    used = M >= 2 * (int64_t)sm_count();
+    if (!used) return cudaSuccess;
+    switch (__builtin_ctz((unsigned)K)) {
+        case 11: return launch_fwht_stream<11, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 12: return launch_fwht_stream<12, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 13: return launch_fwht_stream<13, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 14: return launch_fwht_stream<14, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
+        default: used = false; return cudaSuccess;
+    }
+}
+
 template <class Src>
 cudaError_t dispatch(const Src &src, int64_t M, int K, const float *gain, float eps, int fwht, int mode,
                      int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s) {
     if (fwht) {
+        bool used = false;
+        const cudaError_t e = dispatch_stream(src, M, K, gain, eps, mode, codes, scale_x, zf, s, used);
+        if (used) return e;
         switch (__builtin_ctz((unsigned)K)) {
             case 7: return launch_fwht<7>(src, M, gain, eps, mode, codes, scale_x, zf, s);
             case 8: return launch_fwht<8>(src, M, gain, eps, mode, codes, scale_x, zf, s);

@@ -105,6 +105,28 @@ def test_act_quant_bf16_and_gain(fwht):
     _act_case(3, 1024, fwht, "int4", "f32", True)
 
 
+@pytest.mark.parametrize("K,mode,xdt,gain,M", [
+    (2048, "int8", "f32", False, 300), (4096, "int4", "f32", False, 333), (8192, "int8", "bf16", False, 300),
+    (16384, "int4", "f32", False, 301), (4096, "int8", "bf16", True, 500), (16384, "int8", "f32", True, 297),
+])
+def test_act_quant_fwht_streaming(K, mode, xdt, gain, M):
+    # many tokens (M >= 2 x SMs): the persistent FWHT kernel that TMA-loads token rows into
+    # double-buffered swizzled shared memory; every token checked against the oracle
+    gen = synthetic.generator(K + M)
+    X = synthetic.student_t3((M, K), gen)
+    X[:, synthetic.outlier_channels(K, K // 100, gen)] *= 50.0
+    g = (1.0 + 0.5 * torch.rand(K, generator=gen)) if gain else None
+    if xdt == "bf16":
+        X = X.to(torch.bfloat16)
+    codes, scale = tb.bitnet_act_quant(X.to(DEV), gain=None if g is None else g.to(DEV), fwht=True, mode=mode)
+    X32 = X.float().numpy()
+    gn = None if g is None else g.numpy()
+    q_ref, s_ref = ref.act_quant(X32, gn, 1e-5, True, MODES[mode])
+    sh = ref.shadow(X32, gn, 1e-5, True, MODES[mode])
+    parity.check_codes(host(codes), q_ref, sh, f"stream K={K} {mode} {xdt} gain={gain}")
+    parity.check_scale_bound(host(scale), s_ref, K, MODES[mode], f"stream K={K}")
+
+
 def test_act_quant_many_tokens_flip_rate():
     # 512 tokens x 8192: the flip-rate bound is statistical, so test it on a large sample
     _act_case(512, 8192, True, "int4", "f32", False, seed=11)
