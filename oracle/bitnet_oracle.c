@@ -473,3 +473,106 @@ int oracle_shadow_kv(const float *kv, int64_t BH, int64_t S, int64_t D, int bits
     return ORACLE_OK;
 }
 
+
+/* ---------------------------------------------------------------------------
+ * TL2 weight format (1.67 bits per weight).  [edge] SignedUnsignedWeightPacker and
+ * TL2KernelEdge: the K ternary weights of a row are taken three at a time, triplet
+ * j = (t[3j], t[3j+1], t[3j+2]); element-wise mirror consolidation maps each of the
+ * 27 triplets to a 4-bit index into the 14 "non-negative" base triplets plus a sign
+ * bit (1 = the triplet is the negation of its base).  Read as a balanced-ternary
+ * number, v = 9 t0 + 3 t1 + t2 lies in [-13, 13]; negating the triplet negates v, the
+ * page's base triplets (first nonzero element +1, and the zero triplet) are exactly the
+ * 14 with v >= 0, listed in order of v.  So
+ *   index = |v|,  sign = (v < 0).
+ * Storage (this library's byte layout of the page's two arrays): a row is padded with
+ * zero weights to a multiple of 96 (32 triplets); each group of 32 triplets is 20
+ * bytes: four little-endian 32-bit index words (word i: triplets 8i..8i+7, triplet
+ * 8i + j in bits [4j, 4j+4)) and one little-endian 32-bit sign word (triplet j in bit
+ * j).  Row n starts at byte n * 20 * ceil(K/96).
+ * ------------------------------------------------------------------------- */
+int64_t oracle_tl2_row_bytes(int64_t K) { return K <= 0 ? 0 : 20 * ((K + 95) / 96); }
+
+int oracle_pack_tl2(const int8_t *t, int64_t N, int64_t K, uint8_t *tl2)
+{
+    if (K <= 0 || N < 0) return ORACLE_BAD_ARG;
+    const int64_t rb = oracle_tl2_row_bytes(K), groups = rb / 20;
+    memset(tl2, 0, (size_t)(N * rb));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < groups * 32; ++j) {
+            int w[3];
+            for (int e = 0; e < 3; ++e) {
+                const int64_t k = 3 * j + e;
+                w[e] = k < K ? t[n * K + k] : 0;
+                if (w[e] < -1 || w[e] > 1) return ORACLE_BAD_ARG;
+            }
+            const int v = 9 * w[0] + 3 * w[1] + w[2];
+            const unsigned idx = (unsigned)(v < 0 ? -v : v), sign = v < 0 ? 1u : 0u;
+            uint8_t *grp = tl2 + n * rb + (j / 32) * 20;
+            const int64_t jj = j % 32;
+            const uint32_t word = (uint32_t)idx << (4 * (jj % 8));
+            for (int b = 0; b < 4; ++b) grp[4 * (jj / 8) + b] |= (uint8_t)(word >> (8 * b));
+            grp[16 + jj / 8] |= (uint8_t)(sign << (jj % 8));
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* The triplet of (index, sign), by the definition above; returns 0 for an index > 13. */
+static int tl2_triplet(unsigned idx, unsigned sign, int *w)
+{
+    if (idx > 13) return 0;
+    int v = (int)idx;
+    /* balanced-ternary digits of v in [0, 13]: v = 9 w0 + 3 w1 + w2, digits in {-1, 0, 1} */
+    for (int e = 2; e >= 0; --e) {
+        int d = ((v % 3) + 3) % 3;   /* 0, 1 or 2 */
+        if (d == 2) d = -1;
+        w[e] = d;
+        v = (v - d) / 3;
+    }
+    if (sign)
+        for (int e = 0; e < 3; ++e) w[e] = -w[e];
+    return 1;
+}
+
+int oracle_unpack_tl2(const uint8_t *tl2, int64_t N, int64_t K, int8_t *t)
+{
+    if (K <= 0 || N < 0) return ORACLE_BAD_ARG;
+    const int64_t rb = oracle_tl2_row_bytes(K);
+    int bad = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; k += 3) {
+            const int64_t j = k / 3;
+            const uint8_t *grp = tl2 + n * rb + (j / 32) * 20;
+            const int64_t jj = j % 32;
+            const unsigned idx = (grp[4 * (jj / 8) + (jj % 8) / 2] >> (4 * (jj % 2))) & 15u;
+            const unsigned sign = (grp[16 + jj / 8] >> (jj % 8)) & 1u;
+            int w[3] = {0, 0, 0};
+            if (!tl2_triplet(idx, sign, w)) bad = 1;
+            for (int e = 0; e < 3 && k + e < K; ++e) t[n * K + k + e] = (int8_t)w[e];
+        }
+    }
+    return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
+/* acc[m][n] = sum_k q[m][k] * t[n][k] with each weight read out of the TL2 bytes. */
+int oracle_gemm_tl2(const int8_t *q, const uint8_t *tl2, int64_t M, int64_t N, int64_t K, int32_t *acc)
+{
+    if (K <= 0) return ORACLE_BAD_ARG;
+    const int64_t rb = oracle_tl2_row_bytes(K);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t s = 0;
+            for (int64_t k = 0; k < K; k += 3) {
+                const int64_t j = k / 3;
+                const uint8_t *grp = tl2 + n * rb + (j / 32) * 20;
+                const int64_t jj = j % 32;
+                const unsigned idx = (grp[4 * (jj / 8) + (jj % 8) / 2] >> (4 * (jj % 2))) & 15u;
+                const unsigned sign = (grp[16 + jj / 8] >> (jj % 8)) & 1u;
+                int w[3] = {0, 0, 0};
+                if (!tl2_triplet(idx, sign, w)) return ORACLE_BAD_ARG;
+                for (int e = 0; e < 3 && k + e < K; ++e) s += (int32_t)q[m * K + k + e] * (int32_t)w[e];
+            }
+            acc[m * N + n] = s;
+        }
+    return ORACLE_OK;
+}

@@ -56,10 +56,16 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_shadow_kv.argtypes = [P, I64, I64, I64, I, D, P]
     L.oracle_shadow_swiglu.argtypes = [P, P, I64, I64, P, D, I, I, P]
     L.oracle_round_bf16.argtypes = [P, I64, P]
+    L.oracle_tl2_row_bytes.argtypes = [I64]
+    L.oracle_tl2_row_bytes.restype = I64
+    L.oracle_pack_tl2.argtypes = [P, I64, I64, P]
+    L.oracle_unpack_tl2.argtypes = [P, I64, I64, P]
+    L.oracle_gemm_tl2.argtypes = [P, P, I64, I64, I64, P]
     for name in ("oracle_rmsnorm", "oracle_fwht", "oracle_act_quant", "oracle_shadow_prerounding",
                  "oracle_ternarize", "oracle_pack", "oracle_unpack", "oracle_gemm_int",
                  "oracle_gemm_packed", "oracle_dequant", "oracle_swiglu", "oracle_shadow_swiglu",
-                 "oracle_kv_quant", "oracle_shadow_kv"):
+                 "oracle_kv_quant", "oracle_shadow_kv", "oracle_pack_tl2", "oracle_unpack_tl2",
+                 "oracle_gemm_tl2"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -211,6 +217,39 @@ def unpack(packed, N: int, K: int, L=None) -> np.ndarray:
     t = np.empty((N, K), dtype=np.int8)
     _check("unpack", L.oracle_unpack(_p(packed), N, K, _p(t)))
     return t
+
+
+def tl2_row_bytes(K: int, L=None) -> int:
+    """Bytes of one row in the TL2 format (20 per 32 triplets)."""
+    return int((L or lib()).oracle_tl2_row_bytes(K))
+
+
+def pack_tl2(t, L=None) -> np.ndarray:
+    """Ternary codes [N, K] -> TL2 bytes [N, 20 * ceil(K / 96)] (index and sign planes)."""
+    L = L or lib()
+    t = np.ascontiguousarray(t, dtype=np.int8)
+    N, K = t.shape
+    out = np.empty((N, tl2_row_bytes(K, L)), dtype=np.uint8)
+    _check("pack_tl2", L.oracle_pack_tl2(_p(t), N, K, _p(out)))
+    return out
+
+
+def unpack_tl2(tl2, N: int, K: int, L=None) -> np.ndarray:
+    L = L or lib()
+    tl2 = np.ascontiguousarray(tl2, dtype=np.uint8)
+    t = np.empty((N, K), dtype=np.int8)
+    _check("unpack_tl2", L.oracle_unpack_tl2(_p(tl2), N, K, _p(t)))
+    return t
+
+
+def gemm_tl2(q, tl2, N: int, L=None) -> np.ndarray:
+    L = L or lib()
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    tl2 = np.ascontiguousarray(tl2, dtype=np.uint8)
+    M, K = q.shape
+    acc = np.empty((M, N), dtype=np.int32)
+    _check("gemm_tl2", L.oracle_gemm_tl2(_p(q), _p(tl2), M, N, K, _p(acc)))
+    return acc
 
 
 def pack_weights(W, eps: float = 1e-5, L=None):

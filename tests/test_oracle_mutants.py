@@ -42,6 +42,11 @@ MUTANTS = {
     "kv_step_without_eps": ("float scale = stat + eps;\n        float s = Q / scale;",
                             "float scale = stat;\n        float s = Q / (stat + eps);"),
     "bf16_truncates": ("if (dropped > 0x8000u) r = kept + 1;", "if (0) r = kept + 1;"),
+    "tl2_sign_inverted": ("const unsigned idx = (unsigned)(v < 0 ? -v : v), sign = v < 0 ? 1u : 0u;",
+                          "const unsigned idx = (unsigned)(v < 0 ? -v : v), sign = v > 0 ? 1u : 0u;"),
+    "tl2_digits_reversed": ("v = 9 * w[0] + 3 * w[1] + w[2];", "v = w[0] + 3 * w[1] + 9 * w[2];"),
+    "tl2_sign_word_offset": ("grp[16 + jj / 8] |= (uint8_t)(sign << (jj % 8));",
+                             "grp[12 + jj / 8] |= (uint8_t)(sign << (jj % 8));"),
     "bf16_ties_away": ("else if (dropped == 0x8000u && (kept & 1u)) r = kept + 1;",
                        "else if (dropped == 0x8000u) r = kept + 1;"),
 }

@@ -10,6 +10,8 @@ never against a retyped copy of the oracle's own formulas.
   * Weights: codes in {-1,0,1}; alpha against numpy's float64 mean; the zero
     fraction of Gaussian weights against 2*Phi(sqrt(2/pi)/2) - 1.
   * Packing: hand-worked byte layouts, round trip.
+  * TL2 format: the page's 14 base triplets and their mirrors, hand-worked bytes,
+    every triplet round trip, 5/3 bits per weight, GEMM against numpy.
   * GEMM: numpy int64 matmul.
   * Whole path: the hand-worked tiny cases.
 """
@@ -518,3 +520,70 @@ def test_fwht_gaussianises_heavy_tailed_tokens():
     assert (px > 5 * py).all() and (py < 6).all()       # the outliers are spread over all channels
     # the transform is orthogonal: the mean square (RMSNorm made it 1) is kept
     np.testing.assert_allclose((y.astype(np.float64) ** 2).mean(axis=1), 1.0, rtol=1e-4)
+
+
+# ----------------------------------------------------------------------------- TL2 format
+def _tl2_fields(tl2_row, j):
+    """(index, sign) of triplet j of one TL2 row, read by the documented layout."""
+    grp = tl2_row[(j // 32) * 20:(j // 32) * 20 + 20]
+    jj = j % 32
+    word = int.from_bytes(bytes(grp[4 * (jj // 8):4 * (jj // 8) + 4]), "little")
+    sign = int.from_bytes(bytes(grp[16:20]), "little")
+    return (word >> (4 * (jj % 8))) & 15, (sign >> jj) & 1
+
+
+def test_tl2_base_table_and_mirrors_match_the_page():
+    for idx, trip in _gold("tl2_base_triplets.json")["base"]:
+        for sgn, t in ((0, trip), (1, [-v for v in trip])):
+            row = np.array([t], np.int8)
+            packed = ref.pack_tl2(row)
+            want_sign = sgn if any(trip) else 0
+            assert _tl2_fields(packed[0], 0) == (idx, want_sign), (trip, sgn)
+            np.testing.assert_array_equal(ref.unpack_tl2(packed, 1, 3), row)
+
+
+def test_tl2_layout_golden():
+    for case in _gold("tl2_layout.json")["cases"]:
+        K = case["K"]
+        t = np.zeros((1, K), np.int8)
+        for j, trip in case["triplets"].items():
+            for e, v in enumerate(trip):
+                if 3 * int(j) + e < K:
+                    t[0, 3 * int(j) + e] = v
+        packed = ref.pack_tl2(t)
+        assert packed.tolist() == [case["bytes"]], case["derivation"]
+
+
+def test_tl2_every_triplet_round_trips_and_mirrors():
+    trips = np.array([[a, b, c] for a in (-1, 0, 1) for b in (-1, 0, 1) for c in (-1, 0, 1)], np.int8)  # 27
+    row = trips.reshape(1, -1)
+    packed = ref.pack_tl2(row)
+    np.testing.assert_array_equal(ref.unpack_tl2(packed, 1, row.shape[1]), row)
+    neg = ref.pack_tl2(-row)
+    seen = set()
+    for j in range(27):
+        i1, s1 = _tl2_fields(packed[0], j)
+        i2, s2 = _tl2_fields(neg[0], j)
+        assert i1 == i2 and i1 <= 13
+        assert (s1 ^ s2) == (1 if trips[j].any() else 0)
+        seen.add((i1, s1))
+    assert len(seen) == 27  # the 27 triplets have 27 distinct encodings (14 indices x sign)
+
+
+@pytest.mark.parametrize("N,K", [(5, 96), (7, 100), (3, 4096), (2, 2560), (1, 3)])
+def test_tl2_random_round_trip_and_gemm(N, K):
+    rng = np.random.default_rng(N * 1000 + K)
+    t = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = ref.pack_tl2(t)
+    assert packed.shape == (N, 20 * math.ceil(K / 96))
+    np.testing.assert_array_equal(ref.unpack_tl2(packed, N, K), t)
+    q = rng.integers(-128, 128, size=(4, K)).astype(np.int8)
+    want = q.astype(np.int64) @ t.astype(np.int64).T
+    np.testing.assert_array_equal(ref.gemm_tl2(q, packed, N), want)
+
+
+def test_tl2_is_five_bits_per_three_weights():
+    # the page's 1.67 bits per weight: 4-bit index + 1 sign bit per triplet
+    for K in (96, 960, 6912):
+        assert ref.tl2_row_bytes(K) * 8 / K == pytest.approx(5 / 3)
+    assert ref.tl2_row_bytes(2560) * 8 / 2560 == pytest.approx(20 * 27 * 8 / 2560)  # padded to 2592
