@@ -12,7 +12,9 @@ outlier channels x50, against Wo [4096 x 4096] and Wdown [4096 x 16384]; one ste
 runs the two forwards (1.37 Tera integer ops).  The same line carries a `decode`
 sub-record: the decode configuration (int8 absmax, no FWHT, M in {1, 4, 8} against
 W [6912 x 2560] and [2560 x 6912], six forwards per step) measured the same way with
-its own roofline, step time and CPU baseline.  Inputs are seeded synthetic tensors.
+its own roofline, step time and CPU baseline, and a `decode_tl2` sub-record: the same
+decode configuration with the weights in the TL2 format (5 bits per 3 weights).
+Inputs are seeded synthetic tensors.
 
 Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
 bracketed by a barrier and a device synchronisation, timed with CUDA events on the
@@ -27,8 +29,8 @@ rank time.
 on the same workload, on rank 0 only, each step a bounded sample of tokens and
 output columns extrapolated to the whole step.
 
-Other workloads (--workload): decode, prefill, wdown, wdown_swiglu, msweep_M<M>,
-kvcache.  --out-dtype bf16 stores the forward workloads' outputs in bf16.  Besides
+Other workloads (--workload): decode, decode_tl2, prefill, wdown, wdown_swiglu,
+msweep_M<M>, kvcache.  --out-dtype bf16 stores the forward workloads' outputs in bf16.  Besides
 the contract's keys the line carries `roofline` (the dominant kernel alone, timed in
 one graph over every input rotation), `act_quant` (the activation kernel alone, the
 same way), `e2e`
@@ -64,8 +66,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ----------------------------------------------------------------------------- workloads
 def workload_cases(name: str):
     """(label, M, N, K, mode, fwht, x_kind, x_dtype, outliers) of one step of each workload."""
-    if name == "decode":
-        return [("decode", M, N, K, "int8", False, "normal", "f32", 0)
+    if name in ("decode", "decode_tl2"):
+        return [(name, M, N, K, "int8", False, "normal", "f32", 0)
                 for (N, K) in ((6912, 2560), (2560, 6912)) for M in (1, 4, 8)]
     if name == "prefill":
         cases = []
@@ -86,6 +88,9 @@ def workload_cases(name: str):
 
 
 WORKLOAD_TEXT = {
+    "decode_tl2": "decode GEMV with the weights in the TL2 format (5 bits per 3 weights, mirror-consolidated triplets "
+                  "of the edge page): int8 absmax, no FWHT, X fp32 [M,K] N(0,1), M in {1,4,8}, W [6912x2560] and "
+                  "[2560x6912]; 6 forwards per step",
     "decode": "decode GEMV, int8 absmax, no FWHT: X fp32 [M,K] N(0,1), M in {1,4,8}, against ternary W "
               "[6912x2560] and [2560x6912] (N(0,0.02) absmean-ternarised, 2-bit packed); 6 forwards per step",
     "prefill": "prefill int8, 7B-like projections: X bf16 [4096,4096]; W Wq/Wk/Wv/Wo [4096x4096] (FWHT on Wo only) "
@@ -120,11 +125,13 @@ def make_inputs(cases, seed=0):
     return out
 
 
-def algorithmic_bytes(M, N, K, xdt, out_bytes=4):
-    """Bytes the method must move per forward: X in, codes/scales round trip, packed W, fp32 (or bf16) out."""
+def algorithmic_bytes(M, N, K, xdt, out_bytes=4, weight_bytes=None):
+    """Bytes the method must move per forward: X in, codes/scales round trip, packed W (2 bits per
+    weight unless weight_bytes says otherwise), fp32 (or bf16) out."""
     xb = 2 if xdt == "bf16" else 4
+    wb = N * K // 4 if weight_bytes is None else weight_bytes
     act = M * K * xb + M * K + 4 * M            # act_quant: read X, write codes + scale
-    gemm = N * K // 4 + M * K + 4 * M + out_bytes * M * N + 4  # packed W, codes, scales, out, alpha
+    gemm = wb + M * K + 4 * M + out_bytes * M * N + 4  # packed W, codes, scales, out, alpha
     return act, gemm
 
 
@@ -317,9 +324,10 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
     t_begin = time.perf_counter()
     host = make_inputs(cases)
     packs = []
-    for c in host:
-        packed, alpha, _ = ref.pack_weights(c.W.numpy(), eps=c.eps)
-        packs.append((packed, alpha))
+    tl2 = [c.name.endswith("_tl2") for c in host]
+    for c, is_tl2 in zip(host, tl2):
+        packed, alpha, t = ref.pack_weights(c.W.numpy(), eps=c.eps)
+        packs.append((ref.pack_tl2(t) if is_tl2 else packed, alpha))
     target_step = budget_s / max(4, steps or 4)
     elem_rate = 4e7   # rough single-core rate of the oracle's act_quant (elements/s)
     mac_rate = 2.5e8  # rough single-core rate of the packed-weight loop (MAC/s)
@@ -342,7 +350,10 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
                 X = ref.swiglu(X, c.up[:m].float().numpy())
             q, s_ = ref.act_quant(X, None, c.eps, c.fwht, mode)
             t1 = time.perf_counter()
-            ref.gemm_packed(q, packed[:ncols], ncols)
+            if c.name.endswith("_tl2"):
+                ref.gemm_tl2(q, packed[:ncols], ncols)
+            else:
+                ref.gemm_packed(q, packed[:ncols], ncols)
             t2 = time.perf_counter()
             o = ref.dequant(af, s_, alpha, mode)
             if bf16_out:
@@ -397,6 +408,9 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
     the end-to-end public call.  Returns the rank-local figures."""
     cases = workload_cases(name)
     host = make_inputs(cases)
+    tl2 = name.endswith("_tl2")
+    if tl2 and bf16_out:
+        raise SystemExit("--out-dtype bf16 applies to the 2-bit workloads")
     if bf16_out and any(c.up is not None for c in host):
         raise SystemExit("--out-dtype bf16 applies to the plain forward workloads")
     out_dtype = torch.bfloat16 if bf16_out else torch.float32
@@ -410,7 +424,7 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
         W = c.W.to(dev)
         packed, alpha = tb.bitnet_pack_ternary(W, eps=c.eps)
         del W
-        base.append((packed, alpha))
+        base.append((tb.bitnet_pack_tl2(packed, c.K) if tl2 else packed, alpha))
     packed_bytes = sum(p.numel() for p, _ in base)
 
     def in_bytes(c):
@@ -432,7 +446,9 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
     torch.cuda.synchronize()
 
     def forward(c, X, p, a, out, ws, U):
-        if U is None and bf16_out:
+        if tl2:
+            tb.bitnet_hbitlinear_forward_tl2(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode, out=out, ws=ws)
+        elif U is None and bf16_out:
             tb.bitnet_hbitlinear_forward_ex(X, p, a, c.N, eps=c.eps, fwht=c.fwht, mode=c.mode,
                                             out_dtype=torch.bfloat16, out=out, ws=ws)
         elif U is None:
@@ -499,7 +515,9 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
 
     def gemm_pass(r):
         for c, (codes, scale), (X, p, a, out, ws, U) in zip(host, codes_scales, rot[r]):
-            if bf16_out:
+            if tl2:
+                tb.bitnet_ternary_gemm_tl2(codes, scale, c.mode, p, a, c.N, out=out)
+            elif bf16_out:
                 tb.bitnet_ternary_gemm_ex(codes, scale, c.mode, p, a, c.N, out_dtype=torch.bfloat16, out=out)
             else:
                 tb.bitnet_ternary_gemm(codes, scale, c.mode, p, a, c.N, out=out)
@@ -513,17 +531,19 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
             gemm_pass(r)
     gemm_ms, reps = _timed_graph_replays(torch, gg, stream, sub_s)
     launches = reps * R * len(host)
-    gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32", out_bytes)[1] for c in host)
+    gemm_bytes = reps * R * sum(algorithmic_bytes(c.M, c.N, c.K, "f32", out_bytes, p.numel())[1]
+                                for c, (p, _) in zip(host, base))
     gemm_ops = reps * R * sum(2.0 * c.M * c.N * c.K for c in host)
-    weight_bytes = reps * R * sum(c.N * c.K / 4 for c in host)
+    weight_bytes = reps * R * sum(p.numel() for p, _ in base)
     avg_launch_s = gemm_ms / 1e3 / launches
     if decode_like:
         achieved = gemm_bytes / launches / avg_launch_s / 1e9
         peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic(f"gemv_traffic_{name}", "gemv.cu"),
-                "kernel": "gemv_kernel (register-streamed packed weights, mma.sync s8, in-CTA split-K)",
+                "traffic": profile_traffic(f"gemv_traffic_{name}", "tl2.cu" if tl2 else "gemv.cu"),
+                "kernel": ("gemv_tl2_kernel (TL2 triplets decoded through a 32-entry shared-memory table, mma.sync s8)"
+                           if tl2 else "gemv_kernel (register-streamed packed weights, mma.sync s8, in-CTA split-K)"),
                 "peak_source": f"hbm_gbs of {peak_src} MEASURED_PEAKS.json (copy, burst)",
                 "avg_launch_us": round(avg_launch_s * 1e6, 3),
                 "bytes_per_launch": round(gemm_bytes / launches)}
@@ -627,7 +647,7 @@ def run_ours(args):
 
     m = measure_forward(torch, tb, args.workload, dev, world, args.steps, args.warmup, bf16_out, sampler, stream)
     max_ms, tokens_all = aggregate(m["elapsed_ms"], m["tokens_rank"], world, dev)
-    sub = None
+    sub = sub_tl2 = None
     if args.workload == DEFAULT_WORKLOAD and not args.no_decode_record:
         # the decode configuration, same rules, in the same process: enough steps for
         # about half a second of timed work
@@ -641,6 +661,14 @@ def run_ours(args):
                "act_quant": d["act_quant"], "gpu_launches": d["gpu_launches"],
                "clocks": {k: d["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
                "device_status": d["status"]}
+        # the same decode configuration with the weights in the TL2 format
+        t = measure_forward(torch, tb, "decode_tl2", dev, world, d_steps, args.warmup, False, sampler, stream,
+                            e2e=False)
+        t_ms, t_tok = aggregate(t["elapsed_ms"], t["tokens_rank"], world, dev)
+        sub_tl2 = {"workload": workload_text("decode_tl2"), "name": "decode_tl2", "steps": d_steps,
+                   "value": round(t_tok / (t_ms / 1e3), 1), "unit": "tokens/s",
+                   "ms_per_step": round(t_ms / d_steps, 6), "roofline": t["roofline"],
+                   "gpu_launches": t["gpu_launches"], "device_status": t["status"]}
     sampler.stop()
 
     result = None
@@ -667,6 +695,8 @@ def run_ours(args):
         }
         if sub is not None:
             result["decode"] = sub
+        if sub_tl2 is not None:
+            result["decode_tl2"] = sub_tl2
     # every rank has finished its GPU work; rank 0 now times the oracle on the host (N=1 only)
     if world > 1:
         import torch.distributed as dist
@@ -957,8 +987,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    help=f"{DEFAULT_WORKLOAD} (default) | decode | prefill | wdown | wdown_swiglu | msweep_M<M> | "
-                         "kvcache")
+                    help=f"{DEFAULT_WORKLOAD} (default) | decode | decode_tl2 | prefill | wdown | wdown_swiglu | "
+                         "msweep_M<M> | kvcache")
     ap.add_argument("--no-decode-record", action="store_true",
                     help="skip the decode sub-record of the default workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")

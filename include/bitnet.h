@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define BITNET_ABI_VERSION 7
+#define BITNET_ABI_VERSION 8
 
 #if defined(__GNUC__)
 #define BITNET_API __attribute__((visibility("default")))
@@ -275,6 +275,39 @@ BITNET_API bitnet_status_t bitnet_hbitlinear_forward_noalloc(const void *X, bitn
                                                               bitnet_act_mode_t mode, const uint8_t *packed,
                                                               const float *alpha, int64_t N, float *out,
                                                               void *stream);
+
+/* --------------------------------------------------------------------------
+ * TL2 weight format: 5 bits per 3 weights (1.67 bits per weight), a decode option.
+ * Definition: bitnet_cpp_edge.py page, SignedUnsignedWeightPacker (element-wise mirror
+ * consolidation: 27 ternary triplets -> 14 base triplets + a sign bit) and
+ * TL2KernelEdge.  Triplet j of a row is (t[3j], t[3j+1], t[3j+2]) (weights past K are
+ * 0); read as v = 9 t0 + 3 t1 + t2 in [-13, 13], its index is |v| (the page's base
+ * triplets, first nonzero element +1, in order of v) and its sign is v < 0.
+ * Layout: row n occupies bitnet_tl2_bytes(1, K) = 20 * ceil(K/96) bytes starting at
+ *   n * 20 * ceil(K/96); each group of 32 triplets (96 weights) is 20 bytes: four
+ *   little-endian 32-bit index words (triplet 8i + j of the group in bits [4j, 4j+4) of
+ *   word i) followed by one little-endian 32-bit sign word (triplet j in bit j).
+ * bitnet_pack_tl2: converts 2-bit packed weights (layout above, from
+ *   bitnet_pack_ternary) into this format exactly; alpha is unchanged.  packed
+ *   [N][K/4] read, tl2 [bitnet_tl2_bytes(N, K)] written, both device, 16-byte aligned.
+ * bitnet_ternary_gemm_tl2 / bitnet_hbitlinear_forward_tl2: bitnet_ternary_gemm and
+ *   bitnet_hbitlinear_forward with the weights in this format; decode sizes only:
+ *   M > 16 returns BITNET_ERR_UNSUPPORTED_SHAPE.  Results are identical to the 2-bit
+ *   calls on the same weights (same exact int32 sums, same epilogue).  The decode kernel
+ *   looks each triplet's three signed bytes up in a 32-entry shared-memory table
+ *   (index | sign << 4), so it spends more instructions per weight than the 2-bit
+ *   kernel for 5/6 of its bytes.
+ * ------------------------------------------------------------------------ */
+BITNET_API size_t bitnet_tl2_bytes(int64_t N, int64_t K);
+BITNET_API bitnet_status_t bitnet_pack_tl2(const uint8_t *packed, int64_t N, int64_t K, uint8_t *tl2, void *stream);
+BITNET_API bitnet_status_t bitnet_ternary_gemm_tl2(const int8_t *codes, const float *scale_x, bitnet_act_mode_t mode,
+                                                   const uint8_t *tl2, const float *alpha, int64_t M, int64_t N,
+                                                   int64_t K, float *out, int32_t *acc_out, void *stream);
+BITNET_API bitnet_status_t bitnet_hbitlinear_forward_tl2(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                                         const float *gain, float eps, int fwht,
+                                                         bitnet_act_mode_t mode, const uint8_t *tl2,
+                                                         const float *alpha, int64_t N, float *out, void *ws,
+                                                         size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * bitnet_kv_quant -- the low-bit KV cache of a BitNet v2 attention layer.

@@ -27,7 +27,8 @@ __all__ = [
     "bitnet_get_last_device_status", "bitnet_selftest_wait_timeout", "bitnet_abi_version", "mode_id",
     "bitnet_gemm_token_tile", "bitnet_gemm_force_token_tile", "bitnet_gemm_force_k_splits",
     "bitnet_forward_gemm_plan", "bitnet_workspace_bytes", "bitnet_gemm_workspace_bytes",
-    "bitnet_forward_kernel_count",
+    "bitnet_forward_kernel_count", "bitnet_tl2_bytes", "bitnet_pack_tl2", "bitnet_ternary_gemm_tl2",
+    "bitnet_hbitlinear_forward_tl2",
     "bitnet_act_quant_swiglu", "bitnet_hbitlinear_forward_swiglu", "bitnet_kv_quant",
     "bitnet_ternary_gemm_ex", "bitnet_hbitlinear_forward_ex",
 ]
@@ -349,6 +350,68 @@ def bitnet_hbitlinear_forward_ex(X: torch.Tensor, packed: torch.Tensor, alpha: t
                   L.bitnet_hbitlinear_forward_ex(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)),
                                                  mode_id(mode), _ptr(packed), _ptr(alpha), N, _ptr(out), dt,
                                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def bitnet_tl2_bytes(N: int, K: int) -> int:
+    """Bytes of an N x K weight matrix in the TL2 format (20 per 96 weights of a row)."""
+    return _native.load().bitnet_tl2_bytes(N, K)
+
+
+def bitnet_pack_tl2(packed: torch.Tensor, K: int, tl2=None, stream=None):
+    """2-bit packed weights [N, K/4] -> the TL2 format (5 bits per 3 weights), exactly.
+    Returns uint8 [N, 20 * ceil(K/96)]."""
+    L = _native.load()
+    _need(packed, "packed", torch.uint8)
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError(f"packed must be [N, K/4] = [N, {K // 4}], got {tuple(packed.shape)}")
+    rb = L.bitnet_tl2_bytes(1, K)
+    tl2 = torch.empty((N, rb), dtype=torch.uint8, device=packed.device) if tl2 is None else tl2
+    _need(tl2, "tl2", torch.uint8, (N, rb))
+    _native.check("bitnet_pack_tl2", L.bitnet_pack_tl2(_ptr(packed), N, K, _ptr(tl2), _stream(stream)))
+    return tl2
+
+
+def bitnet_ternary_gemm_tl2(codes: torch.Tensor, scale_x: torch.Tensor, mode, tl2: torch.Tensor,
+                            alpha: torch.Tensor, N: int, out=None, acc_out=None, stream=None):
+    """bitnet_ternary_gemm with TL2 weights (M <= 16).  Returns out fp32 [M, N]."""
+    L = _native.load()
+    _need(codes, "codes", torch.int8)
+    M, K = codes.shape
+    _need(scale_x, "scale_x", torch.float32, (M,))
+    _need(tl2, "tl2", torch.uint8, (N, L.bitnet_tl2_bytes(1, K)))
+    _need(alpha, "alpha", torch.float32)
+    out = torch.empty((M, N), dtype=torch.float32, device=codes.device) if out is None else out
+    _need(out, "out", torch.float32, (M, N))
+    if acc_out is not None:
+        _need(acc_out, "acc_out", torch.int32, (M, N))
+    _native.check("bitnet_ternary_gemm_tl2",
+                  L.bitnet_ternary_gemm_tl2(_ptr(codes), _ptr(scale_x), mode_id(mode), _ptr(tl2), _ptr(alpha), M, N,
+                                            K, _ptr(out), _ptr(acc_out), _stream(stream)))
+    return out
+
+
+def bitnet_hbitlinear_forward_tl2(X: torch.Tensor, tl2: torch.Tensor, alpha: torch.Tensor, N: int, gain=None,
+                                  eps: float = 1e-5, fwht: bool = True, mode="int8", out=None, ws=None,
+                                  stream=None):
+    """The whole H-BitLinear forward with TL2 weights (M <= 16).  Returns out fp32 [M, N]."""
+    L = _native.load()
+    _need(X, "X")
+    M, K = X.shape
+    _need(tl2, "tl2", torch.uint8, (N, L.bitnet_tl2_bytes(1, K)))
+    _need(alpha, "alpha", torch.float32)
+    if gain is not None:
+        _need(gain, "gain", torch.float32, (K,))
+    out = torch.empty((M, N), dtype=torch.float32, device=X.device) if out is None else out
+    _need(out, "out", torch.float32, (M, N))
+    nbytes = L.bitnet_forward_workspace_bytes(M, K)
+    ws = torch.empty((max(nbytes, 256),), dtype=torch.uint8, device=X.device) if ws is None else ws
+    _need(ws, "ws", torch.uint8)
+    _native.check("bitnet_hbitlinear_forward_tl2",
+                  L.bitnet_hbitlinear_forward_tl2(_ptr(X), _xdt(X), M, K, _ptr(gain), eps, int(bool(fwht)),
+                                                  mode_id(mode), _ptr(tl2), _ptr(alpha), N, _ptr(out), _ptr(ws),
+                                                  ws.numel(), _stream(stream)))
     return out
 
 

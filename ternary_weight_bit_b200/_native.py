@@ -61,6 +61,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
         "bitnet_workspace_bytes": (SZ, [I64, I64, I64]),
         "bitnet_forward_kernel_count": (I, [I64, I64, I64, I, I]),
+        "bitnet_tl2_bytes": (SZ, [I64, I64]),
+        "bitnet_pack_tl2": (I, [P, I64, I64, P, P]),
+        "bitnet_ternary_gemm_tl2": (I, [P, P, I, P, P, I64, I64, I64, P, P, P]),
+        "bitnet_hbitlinear_forward_tl2": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P, SZ, P]),
         "bitnet_forward_workspace_bytes": (SZ, [I64, I64]),
         "bitnet_hbitlinear_forward": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P, SZ, P]),
         "bitnet_hbitlinear_forward_noalloc": (I, [P, I, I64, I64, P, F, I, I, P, P, I64, P, P]),

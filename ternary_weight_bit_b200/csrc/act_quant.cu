@@ -254,6 +254,9 @@ __device__ __forceinline__ void fwht_quant_token(float (&v)[FwhtShape<LOGK>::E],
     constexpr int W = T / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row = token * K;
+    // Materialise the partial sum now: left to itself the compiler sinks its products
+    // to the reduction at the end and keeps the E inputs alive through the transform.
+    asm volatile("" : "+f"(ss));
 
     if (gain != nullptr) {
 #pragma unroll

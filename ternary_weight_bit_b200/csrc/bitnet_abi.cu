@@ -381,6 +381,47 @@ bitnet_status_t bitnet_hbitlinear_forward_swiglu(const void *gate, const void *u
     return forward_ws(gate, up, xdt, M, K, gain, eps, fwht, mode, packed, alpha, N, out, false, ws, ws_bytes, stream);
 }
 
+size_t bitnet_tl2_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K <= 0) return 0;
+    return (size_t)N * tl2_row_bytes(K);
+}
+
+bitnet_status_t bitnet_pack_tl2(const uint8_t *packed, int64_t N, int64_t K, uint8_t *tl2, void *stream) {
+    if (N < 1 || N > kMaxRows) return BITNET_ERR_INVALID_ARG;
+    bitnet_status_t st = check_k(K, 0);
+    if (st != BITNET_OK) return st;
+    if (!packed || !tl2 || !aligned16(packed) || !aligned16(tl2)) return BITNET_ERR_INVALID_ARG;
+    return from_cuda(launch_tl2_pack(packed, N, (int)K, tl2, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status_t bitnet_ternary_gemm_tl2(const int8_t *codes, const float *scale_x, bitnet_act_mode_t mode,
+                                        const uint8_t *tl2, const float *alpha, int64_t M, int64_t N, int64_t K,
+                                        float *out, int32_t *acc_out, void *stream) {
+    bitnet_status_t st = validate_gemm(codes, scale_x, mode, tl2, alpha, M, N, K, out, acc_out);
+    if (st != BITNET_OK || M == 0) return st;
+    if (M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED_SHAPE;  // a decode format
+    return from_cuda(launch_gemv_tl2(codes, scale_x, mode, tl2, alpha, (int)M, (int)N, (int)K, out, acc_out, true,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status_t bitnet_hbitlinear_forward_tl2(const void *X, bitnet_dtype_t xdt, int64_t M, int64_t K,
+                                              const float *gain, float eps, int fwht, bitnet_act_mode_t mode,
+                                              const uint8_t *tl2, const float *alpha, int64_t N, float *out,
+                                              void *ws, size_t ws_bytes, void *stream) {
+    bitnet_status_t st = validate_forward(X, xdt, M, K, gain, fwht, mode, tl2, alpha, N, out);
+    if (st != BITNET_OK || M == 0) return st;
+    if (M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED_SHAPE;
+    if (!ws || ws_bytes < bitnet_forward_workspace_bytes(M, K) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return BITNET_ERR_WORKSPACE;
+    int8_t *codes = static_cast<int8_t *>(ws);
+    float *scale_x = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256((size_t)M * (size_t)K));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_act_quant(X, xdt == BITNET_BF16, M, (int)K, gain, eps, fwht, mode, codes, scale_x, s);
+    if (e == cudaSuccess)
+        e = launch_gemv_tl2(codes, scale_x, mode, tl2, alpha, (int)M, (int)N, (int)K, out, nullptr, true, s);
+    return from_cuda(e);
+}
+
 int bitnet_gemm_token_tile(int64_t M, int64_t N, int64_t K) {
     if (M < 0 || N < 1 || N > kMaxRows || check_k(K, 0) != BITNET_OK) return -1;
     if (M <= kGemvMaxM) return 0;

@@ -16,7 +16,8 @@ PKG = os.path.dirname(CSRC)
 ROOT = os.path.dirname(PKG)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbitnet.so")
-SOURCES = ["act_quant.cu", "pack.cu", "gemv.cu", "gemm_sm100.cu", "kv_quant.cu", "bitnet_abi.cu", "forward_noalloc.cu"]
+SOURCES = ["act_quant.cu", "pack.cu", "gemv.cu", "gemm_sm100.cu", "kv_quant.cu", "tl2.cu", "bitnet_abi.cu",
+           "forward_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
                      "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]

@@ -62,6 +62,14 @@ cudaError_t launch_gemv(const int8_t *codes, const float *scale_x, int mode, con
                         const float *alpha, int M, int N, int K, void *out, int32_t *acc_out,
                         bool pdl, cudaStream_t s, bool out_bf16 = false);
 
+// TL2 format (1.67 bits per weight): bytes per row, the conversion from the 2-bit
+// packed layout (exact) and the decode kernel (M <= 16; out fp32, or bf16 when out_bf16).
+size_t tl2_row_bytes(int64_t K);
+cudaError_t launch_tl2_pack(const uint8_t *packed, int64_t N, int K, uint8_t *tl2, cudaStream_t s);
+cudaError_t launch_gemv_tl2(const int8_t *codes, const float *scale_x, int mode, const uint8_t *tl2,
+                            const float *alpha, int M, int N, int K, void *out, int32_t *acc_out, bool pdl,
+                            cudaStream_t s, bool out_bf16 = false);
+
 // Prefill path: tcgen05 int8 tensor-core GEMM with TMEM accumulators.
 // A plan is a token-tile size (256/224/192/128/64) and a k-split count (1, 2, 4, 8).
 // With splits > 2, `out` must be zero on entry (the kernel adds int32 partial sums

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.bitnet_abi_version() == 7
+    assert L.bitnet_abi_version() == 8
     for s in range(7):
         assert L.bitnet_status_string(s)
     assert L.bitnet_status_string(5).decode().startswith("a kernel gave up")
@@ -162,6 +162,21 @@ def test_forward_kernel_count(L):
     assert L.bitnet_forward_kernel_count(0, 4096, 4096, 0, 0) == 0
     assert L.bitnet_forward_kernel_count(4, 4096, 2560, 1, 0) == -1     # FWHT needs a power of two
     assert L.bitnet_forward_kernel_count(4, 0, 4096, 0, 0) == -1
+
+
+def test_tl2_host_logic(L):
+    # 20 bytes per 96 weights of a row; decode sizes only; the usual argument checks
+    assert L.bitnet_tl2_bytes(1, 96) == 20 and L.bitnet_tl2_bytes(3, 2560) == 3 * 20 * 27
+    assert L.bitnet_tl2_bytes(1, 6912) * 8 / 6912 == pytest.approx(5 / 3)
+    s = P(0)
+    assert L.bitnet_ternary_gemm_tl2(FAKE, FAKE, 0, FAKE, FAKE, 17, 256, 256, FAKE, None, s) == \
+        _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_ternary_gemm_tl2(FAKE, FAKE, 0, FAKE, FAKE, 4, 256, 100, FAKE, None, s) == \
+        _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_hbitlinear_forward_tl2(FAKE, 0, 32, 256, None, 1e-5, 0, 0, FAKE, FAKE, 64, FAKE, FAKE, 1 << 20,
+                                           s) == _native.ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_pack_tl2(FAKE, 16, 256, P(4100), s) == _native.ERR_INVALID_ARG
+    assert L.bitnet_ternary_gemm_tl2(None, None, 0, None, None, 0, 16, 256, None, None, s) == _native.OK
 
 
 def test_gemm_workspace_validation(L):

@@ -242,6 +242,65 @@ def test_gemv_decode_kernel_shapes(M, N, K):
     np.testing.assert_array_equal(parity.bf16_bits(outh), ref.round_bf16(out_ref))
 
 
+# ----------------------------------------------------------------------------- TL2 format
+@pytest.mark.parametrize("N,K", [(256, 256), (300, 384), (6912, 2560), (2560, 6912), (37, 128)])
+def test_pack_tl2_matches_oracle(N, K):
+    # the 2-bit -> TL2 conversion gives the oracle's bytes for the same ternary codes
+    W = synthetic.gaussian((N, K), 0.02, synthetic.generator(N + K))
+    packed, alpha = tb.bitnet_pack_ternary(W.to(DEV))
+    tl2 = tb.bitnet_pack_tl2(packed, K)
+    p_ref, a_ref, t_ref = ref.pack_weights(W.numpy())
+    np.testing.assert_array_equal(host(packed), p_ref)
+    np.testing.assert_array_equal(host(tl2), ref.pack_tl2(t_ref))
+    assert tl2.numel() * 8 / (N * K) == pytest.approx(20 * 8 * math.ceil(K / 96) / K)
+
+
+TL2_SHAPES = [(1, 64, 128), (3, 100, 384), (8, 6912, 2560), (8, 2560, 6912), (16, 512, 1024), (13, 37, 2944),
+              (5, 4096, 16384)]
+
+
+@pytest.mark.parametrize("M,N,K", TL2_SHAPES)
+@pytest.mark.parametrize("mode", ["int8", "int4"])
+def test_gemm_tl2_exact_accumulators(M, N, K, mode):
+    # the TL2 decode kernel: exact int32 sums (oracle reading the TL2 bytes, and the same
+    # sums as the 2-bit format), outputs from the same epilogue
+    q, packed, scale, alpha = _gemm_case(M, N, K, mode, seed=M * 7 + N + K + 5)
+    tl2 = tb.bitnet_pack_tl2(dev(packed), K)
+    acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    out = tb.bitnet_ternary_gemm_tl2(dev(q), dev(scale), mode, tl2, dev(alpha), N, acc_out=acc)
+    acc_ref = ref.gemm_tl2(q, host(tl2), N)
+    np.testing.assert_array_equal(acc_ref, ref.gemm_packed(q, packed, N))
+    np.testing.assert_array_equal(host(acc), acc_ref, err_msg=f"{M}x{N}x{K}")
+    np.testing.assert_array_equal(host(out), ref.dequant(acc_ref, scale, alpha[0], MODES[mode]))
+
+
+@pytest.mark.parametrize("M,NK,fwht,mode", [(1, (6912, 2560), False, "int8"), (8, (2560, 6912), False, "int8"),
+                                            (4, (4096, 4096), True, "int4"), (16, (1000, 1024), True, "int8")])
+def test_forward_tl2_equals_the_2bit_forward(M, NK, fwht, mode):
+    # the same weights in either format give bit-identical forwards, and the forward
+    # matches the oracle end to end
+    N, K = NK
+    case = synthetic.make_case("tl2_fwd", M, K, N, x_kind="student_t3", outliers=max(1, K // 100), outlier_gain=50.0,
+                               fwht=fwht, mode=mode, seed=M + N)
+    Xd = case.X.to(DEV)
+    packed, alpha = tb.bitnet_pack_ternary(case.W.to(DEV))
+    tl2 = tb.bitnet_pack_tl2(packed, K)
+    ws = torch.empty((tb.bitnet_forward_workspace_bytes(M, K),), dtype=torch.uint8, device=DEV)
+    out_tl2 = tb.bitnet_hbitlinear_forward_tl2(Xd, tl2, alpha, N, fwht=fwht, mode=mode, ws=ws)
+    gcodes, gs = (host(a) for a in ws_codes_scales(ws, M, K))
+    out_2bit = tb.bitnet_hbitlinear_forward(Xd, packed, alpha, N, fwht=fwht, mode=mode)
+    torch.cuda.synchronize()
+    assert torch.equal(out_tl2, out_2bit)
+    X32 = case.X.numpy()
+    p_ref, a_ref, _ = ref.pack_weights(case.W.numpy())
+    m = MODES[mode]
+    r = ref.hbitlinear_forward(X32, p_ref, a_ref, N, fwht_on=fwht, mode=m)
+    parity.check_codes(gcodes, r.codes, ref.shadow(X32, None, 1e-5, fwht, m), "tl2 forward")
+    parity.check_out_same_codes(host(out_tl2), ref.dequant(ref.gemm_tl2(gcodes, ref.pack_tl2(ref.unpack(p_ref, N, K)),
+                                                                        N), gs, a_ref, m), "tl2 forward")
+    parity.check_out_end_to_end(host(out_tl2), r.out, gcodes, r.codes, r.scale_x, a_ref, m, "tl2 forward")
+
+
 def test_gemm_extreme_codes():
     # every code at the int8 extremes, every weight +1/-1: |acc| = 128 K is the largest possible
     for M, N, K in [(4, 64, 16384), (32, 256, 16384)]:
