@@ -63,14 +63,18 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 // ------------------------------------------------------------------ quantiser
-// Round-clip y*s to [lo, hi] with round-half-to-even: adding 1.5*2^23 rounds an fp32
-// in [-2^22, 2^22] to the nearest integer (ties to even) and leaves that integer in
-// the low mantissa bits.  Returns the whole word (code in the low byte); clips only
-// when asked.
+// Round-clip y*s to [lo, hi] with round-half-to-even in one fused multiply-add:
+// y*s + 1.5*2^23, rounded once, is 1.5*2^23 plus the integer nearest the exact product
+// (ties to even) while |y*s| < 2^22, that integer sitting in the low mantissa bits.
+// The clip acts on the biased value (an integer in [lo, hi] then), which also holds any
+// larger |y*s| at the bound.  Returns the whole word (code in the low byte); clips only
+// when asked.  Against rounding the product first, the code can change only where the
+// exact product lies within half an ulp of a rounding tie.
 __device__ __forceinline__ uint32_t quant_bits(float y, float s, float lo, float hi, bool clip) {
-    float v = __fmul_rn(y, s);
-    if (clip) v = fminf(fmaxf(v, lo), hi);
-    return __float_as_uint(__fadd_rn(v, 12582912.0f));
+    constexpr float kBias = 12582912.0f;  // 1.5 * 2^23
+    float v = __fmaf_rn(y, s, kBias);
+    if (clip) v = fminf(fmaxf(v, kBias + lo), kBias + hi);
+    return __float_as_uint(v);
 }
 
 // Low bytes of four words -> one word (byte permutes).
