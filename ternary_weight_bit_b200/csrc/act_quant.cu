@@ -124,6 +124,14 @@ __device__ __forceinline__ void load8(const void *X, int64_t idx, float *v) {
 }
 
 template <bool BF16>
+__device__ __forceinline__ float load1(const void *X, int64_t idx) {
+    if constexpr (BF16)
+        return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(X) + idx) << 16);
+    else
+        return __ldg(reinterpret_cast<const float *>(X) + idx);
+}
+
+template <bool BF16>
 __device__ __forceinline__ void load4(const void *X, int64_t idx, float *v) {
     if constexpr (BF16) {
         const uint2 u = __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const uint16_t *>(X) + idx));
@@ -147,6 +155,7 @@ struct XSrc {
     const void *X;
     __device__ __forceinline__ void get8(int64_t idx, float *v) const { load8<BF16>(X, idx, v); }
     __device__ __forceinline__ void get4(int64_t idx, float *v) const { load4<BF16>(X, idx, v); }
+    __device__ __forceinline__ float get1(int64_t idx) const { return load1<BF16>(X, idx); }
     // L2 prefetch of n elements from idx (a hint: it returns no data, so it is safe before
     // the dependency wait -- L2 is where every write lands, so what is read later is current)
     __device__ __forceinline__ void prefetch(int64_t idx, int n) const {
@@ -172,6 +181,9 @@ struct SwigluSrc {
         load8<BF16>(up, idx, u);
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = swiglu(v[i], u[i]);
+    }
+    __device__ __forceinline__ float get1(int64_t idx) const {
+        return swiglu(load1<BF16>(gate, idx), load1<BF16>(up, idx));
     }
     __device__ __forceinline__ void get4(int64_t idx, float *v) const {
         float u[4];
@@ -410,112 +422,204 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
 }
 
 // ------------------------------------------------------------------ streaming FWHT kernel
-// For many tokens: a persistent grid whose CTAs loop over tokens (t = blockIdx.x,
-// + gridDim.x, ...).  Each token row is brought into shared memory by TMA tensor copies
-// (X viewed as [M][K/32][32], boxes of up to 256 rows of 32 elements, 128-byte (fp32)
-// or 64-byte (bf16) swizzled).  The copy of the CTA's next token is issued as soon as
-// every thread has read the current one (after the first transpose), so its HBM latency
-// overlaps the rest of the transform; one buffer per CTA keeps several CTAs resident
-// per SM.  The swizzle lets thread tid read its 32 contiguous elements (row tid of the
-// buffer) with 16-byte loads free of bank conflicts.  The transform is fwht_quant_token.
-template <int LOGK, bool BF16>
+// For many tokens with 2^11 <= K <= 2^14: a persistent grid whose CTAs loop over tokens
+// (t = blockIdx.x, + gridDim.x, ...), several CTAs resident per SM.  The transform takes
+// two register phases and one shared-memory transpose.  With ELOG = ceil(LOGK/2)
+// register bits and TLOG = LOGK - ELOG thread bits per phase:
+//   phase 0: thread t holds elements t + (r << TLOG), r < 2^ELOG, so each load
+//            instruction of a warp reads 32 consecutive elements, and runs the
+//            butterflies of element bits TLOG..LOGK-1;
+//   phase 1: thread t holds the 2^ELOG consecutive elements t*2^ELOG + r, read back as
+//            16-byte units, and runs the butterflies of bits 0..TLOG-1 (for odd LOGK,
+//            bit TLOG rides along untouched); its codes leave as 16-byte stores.
+// Element i sits in shared memory at word i ^ (((i >> ELOG) & 7) << 2): the 16-byte unit
+// index is XORed with three bits of the element's phase-1 owner, which keeps both the
+// phase-0 word stores and the phase-1 16-byte loads free of bank conflicts.  The
+// butterflies run on register pairs with the packed fp32 add and fma of sm_100 (a - b as
+// fma(b, -1, a): the same single rounding as a subtraction), except in the register bit
+// that forms the pairs.  The bits are transformed in another order than in the per-token
+// kernel, so results differ from it in the last bits only.  Each token's row is prefetched
+// into L2 two tokens ahead; the barriers per token are two: after the transpose's stores,
+// and in the statistic's reduction, whose result every thread then finishes itself.
+template <int LOGK>
 struct StreamShape {
-    using S = FwhtShape<LOGK>;
-    static constexpr int K = S::K;
-    static constexpr int ROWS = K / 32;                         // 32-element rows per token
-    static constexpr int BOX = ROWS < 256 ? ROWS : 256;        // rows per TMA box
-    static constexpr int NBOX = ROWS / BOX;
-    static constexpr int XBYTES = K * (BF16 ? 2 : 4);          // one token row
-    static constexpr int TBYTES = (K + K / 32) * 4;            // transpose buffer
-    static constexpr int SMEM = XBYTES + TBYTES + 1024;        // + 1024-byte alignment
+    static constexpr int K = 1 << LOGK;
+    static constexpr int ELOG = (LOGK + 1) / 2;
+    static constexpr int E = 1 << ELOG;       // elements per thread
+    static constexpr int TLOG = LOGK - ELOG;
+    static constexpr int T = 1 << TLOG;       // threads per CTA
+    static constexpr int W = T / 32;
+    static constexpr int MINB = (E >= 128 ? 384 : 512) / T;  // CTAs per SM the registers allow
+    static constexpr int SMEM = K * 4;
 };
 
-template <int LOGK, bool BF16>
-__global__ void __launch_bounds__(FwhtShape<LOGK>::T)
-act_quant_fwht_stream_kernel(const __grid_constant__ CUtensorMap tmx, const float *__restrict__ gain, float eps,
-                             int mode, int64_t M, int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf,
-                             int *status, const void *X) {
-    using S = FwhtShape<LOGK>;
-    using SS = StreamShape<LOGK, BF16>;
-    constexpr int E = S::E;
-    static_assert(E == 32, "one 32-element row per thread");
-    extern __shared__ uint8_t smraw[];
-    uint8_t *xbuf = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-    float *sm = reinterpret_cast<float *>(xbuf + SS::XBYTES);  // transpose buffer
-    __shared__ float2 red[32];
-    __shared__ FwhtScalars sc;
-    __shared__ __align__(8) uint64_t full;
-    const int tid = threadIdx.x;
-
-    auto issue = [&](int64_t token) {  // thread 0: the whole row of `token` into the buffer
-        const uint32_t bar = smem_u32(&full);
-        asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-                     "r"((uint32_t)SS::XBYTES)
-                     : "memory");
+// Butterflies of register bit b over E values held as E/2 pairs (pair j = registers 2j, 2j+1).
+template <int NP>
+__device__ __forceinline__ void butterfly_pairs(float2 (&v)[NP], int b) {
+    if (b == 0) {
 #pragma unroll
-        for (int j = 0; j < SS::NBOX; ++j)
-            asm volatile(
-                "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
-                "[%2];" ::"r"(smem_u32(xbuf + j * SS::BOX * (BF16 ? 64 : 128))),
-                "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(bar), "r"(0), "r"(j * SS::BOX), "r"((int)token)
-                : "memory");
-    };
+        for (int j = 0; j < NP; ++j) {
+            const float a = v[j].x, c = v[j].y;
+            v[j] = make_float2(__fadd_rn(a, c), __fsub_rn(a, c));
+        }
+    } else {
+        const int h = 1 << (b - 1);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            if ((j & h) == 0) {
+                const float2 a = v[j], c = v[j | h];
+                v[j] = __fadd2_rn(a, c);
+                v[j | h] = __ffma2_rn(c, make_float2(-1.0f, -1.0f), a);
+            }
+        }
+    }
+}
+
+template <int LOGK, class Src>
+__global__ void __launch_bounds__(StreamShape<LOGK>::T, StreamShape<LOGK>::MINB)
+act_quant_fwht_stream_kernel(Src src, const float *__restrict__ gain, float eps, int mode, int64_t M,
+                             int8_t *__restrict__ codes, float *__restrict__ scale_x, ZeroFill zf) {
+    using S = StreamShape<LOGK>;
+    constexpr int K = S::K, E = S::E, NP = E / 2, ELOG = S::ELOG, TLOG = S::TLOG, W = S::W;
+    extern __shared__ __align__(16) float buf[];  // K floats, swizzled
+    __shared__ float2 red[W];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool mean = mode != BITNET_ACT_INT8_ABSMAX;
+    constexpr float kBias = 12582912.0f;  // 1.5 * 2^23, see quant_bits
+    const float qlo = kBias + (mean ? -8.0f : -128.0f), qhi = kBias + (mean ? 7.0f : 127.0f);
+    const float p2 = __int_as_float((127 - LOGK / 2) << 23);  // 2^(-floor(LOGK/2)), exact
+    const float hs = (LOGK & 1) ? __fmul_rn(0.70710678118654752f, p2) : p2;
+
+    // X may come from the previous kernel: before the dependency wait only warm L2
     if (tid == 0) {
-        mbar_init(&full, 1);
-        fence_mbar_init();
-        tma_prefetch_desc(&tmx);
-        // X may come from the previous kernel: before the dependency wait only warm L2
         for (int i = 0; i < 2; ++i) {
             const int64_t t = blockIdx.x + (int64_t)i * gridDim.x;
-            if (t < M) bulk_prefetch_l2(reinterpret_cast<const uint8_t *>(X) + t * SS::XBYTES, SS::XBYTES);
+            if (t < M) src.prefetch(t * K, K);
         }
     }
     pdl_launch_dependents();
     pdl_wait_prerequisites();
-    __syncthreads();  // the barrier is initialised
-    if (tid == 0) issue(blockIdx.x);
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < M; t += gridDim.x, ++it) {
+
+    for (int64_t t = blockIdx.x; t < M; t += gridDim.x) {
+        if (tid == 0 && t + 2 * (int64_t)gridDim.x < M) src.prefetch((t + 2 * (int64_t)gridDim.x) * K, K);
         zero_fill(zf, t);  // a following split-K GEMM's output row (and, for token 0, its counters)
-        // bounded; on a timeout (recorded in the status word) the loop runs on, so that
-        // every thread still meets every barrier
-        mbar_wait(&full, (uint32_t)it & 1u, status);
-        // row tid of the buffer: 16-byte units swizzled by the row's position in its 1 KB block
-        float v[E];
-        if constexpr (BF16) {
+        const int64_t row = t * K;
+
+        // phase 0: elements tid + (r << TLOG), pairs (2j, 2j+1)
+        float2 v[NP];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(xbuf + tid * 64 + ((u ^ ((tid >> 1) & 3)) << 4));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int j = 0; j < NP; ++j) {
+            v[j].x = src.get1(row + tid + ((2 * j) << TLOG));
+            v[j].y = src.get1(row + tid + ((2 * j + 1) << TLOG));
+        }
+        float2 sa = make_float2(0.0f, 0.0f), sb = sa;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    v[8 * u + 2 * i] = __uint_as_float(ww[i] << 16);
-                    v[8 * u + 2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u);
-                }
-            }
-        } else {
+        for (int j = 0; j < NP; j += 2) {
+            sa = __ffma2_rn(v[j], v[j], sa);
+            sb = __ffma2_rn(v[j + 1], v[j + 1], sb);
+        }
+        float ss = __fadd_rn(__fadd_rn(sa.x, sa.y), __fadd_rn(sb.x, sb.y));
+        asm volatile("" : "+f"(ss));  // keep the sum here, not sunk to its use after phase 1
+        if (gain != nullptr) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float4 w = *reinterpret_cast<const float4 *>(xbuf + tid * 128 + ((u ^ (tid & 7)) << 4));
-                v[4 * u] = w.x;
-                v[4 * u + 1] = w.y;
-                v[4 * u + 2] = w.z;
-                v[4 * u + 3] = w.w;
+            for (int j = 0; j < NP; ++j) {
+                v[j].x = __fmul_rn(v[j].x, __ldg(gain + tid + ((2 * j) << TLOG)));
+                v[j].y = __fmul_rn(v[j].y, __ldg(gain + tid + ((2 * j + 1) << TLOG)));
             }
         }
-        float ss = 0.0f;
 #pragma unroll
-        for (int r = 0; r < E; ++r) ss = fmaf(v[r], v[r], ss);
-        const int64_t next = t + gridDim.x;
-        fwht_quant_token<LOGK>(v, ss, t, gain, eps, mode, codes, scale_x, sm, red, &sc, [&]() {
-            // every thread has read the buffer (the first transpose's barrier): refill it
-            if (tid == 0 && next < M) {
-                fence_proxy_async_smem();  // the reads are ordered before the copy's writes
-                issue(next);
+        for (int b = 0; b < ELOG; ++b) butterfly_pairs(v, b);
+
+        // transpose: word stores in the phase-0 layout, 16-byte loads in the phase-1 layout
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int r = 2 * j + k;
+                // bits ELOG..ELOG+2 of element tid + (r << TLOG) are bits of r (TLOG >= 5)
+                const int sw = ((r << TLOG) >> ELOG) & 7;
+                buf[(tid ^ (sw << 2)) + (r << TLOG)] = k ? v[j].y : v[j].x;
             }
-        });
+        }
+        __syncthreads();
+        const float *rb = buf + tid * E;
+#pragma unroll
+        for (int u = 0; u < E / 4; ++u) {
+            const float4 q = *reinterpret_cast<const float4 *>(rb + 4 * ((u & ~7) | ((u ^ tid) & 7)));
+            v[2 * u] = make_float2(q.x, q.y);
+            v[2 * u + 1] = make_float2(q.z, q.w);
+        }
+#pragma unroll
+        for (int b = 0; b < TLOG; ++b) butterfly_pairs(v, b);
+
+        // one reduction of (sum x^2, max|z| or sum|z|); every thread finishes it
+        float st;
+        if (mean) {
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                a0 += fabsf(v[j].x);
+                a1 += fabsf(v[j].y);
+            }
+            st = a0 + a1;
+        } else {
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                a0 = fmaxf(a0, fabsf(v[j].x));
+                a1 = fmaxf(a1, fabsf(v[j].y));
+            }
+            st = fmaxf(a0, a1);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float x = __shfl_xor_sync(0xffffffffu, st, o);
+            st = mean ? st + x : fmaxf(st, x);
+        }
+        if constexpr (W > 1) {
+            // red was last read before this token's transpose barrier
+            if (lane == 0) red[warp] = make_float2(ss, st);
+            __syncthreads();
+            float2 q = red[0];
+#pragma unroll
+            for (int w = 1; w < W; ++w) {
+                const float2 p = red[w];
+                q.x += p.x;
+                q.y = mean ? q.y + p.y : fmaxf(q.y, p.y);
+            }
+            ss = q.x;
+            st = q.y;
+        }
+        const float rho = __fmul_rn(rms_factor(ss, K, eps), hs);
+        const float rs = __fmul_rn(rho, st);
+        const float stat = mean ? __fdiv_rn(rs, (float)K) : rs;
+        const float s_eff = __fmul_rn(rho, quant_params(stat, eps, mode).s);
+        if (tid == 0) scale_x[t] = stat;
+
+        // codes: rne(z * s_eff) by one fused multiply-add with the rounding bias (see
+        // quant_bits); int4 clips the biased value, int8 never needs to
+        int8_t *out = codes + row + tid * E;
+        const float2 s2 = make_float2(s_eff, s_eff), b2 = make_float2(kBias, kBias);
+#pragma unroll
+        for (int u = 0; u < E / 16; ++u) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 a = __ffma2_rn(v[8 * u + 2 * k], s2, b2);
+                float2 c = __ffma2_rn(v[8 * u + 2 * k + 1], s2, b2);
+                if (mean) {
+                    a.x = fminf(fmaxf(a.x, qlo), qhi);
+                    a.y = fminf(fmaxf(a.y, qlo), qhi);
+                    c.x = fminf(fmaxf(c.x, qlo), qhi);
+                    c.y = fminf(fmaxf(c.y, qlo), qhi);
+                }
+                w[k] = pack4_perm(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(c.x),
+                                  __float_as_uint(c.y));
+            }
+            *reinterpret_cast<uint4 *>(out + 16 * u) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
-    // every copy issued above was waited for in the loop before the CTA exits
 }
 
 // ------------------------------------------------------------------ plain kernel (no FWHT)
@@ -709,34 +813,29 @@ cudaError_t launch_fwht(const Src &src, int64_t M, const float *gain, float eps,
     return launch_pdl(kern, dim3((unsigned)M), dim3(S::T), smem, s, src, gain, eps, mode, codes, scale_x, zf);
 }
 
-// The streaming kernel for K = 2^LOGK, 11 <= LOGK <= 14 (T >= 64 threads, so that the
-// statistic's block reduction has barriers; two rows and the transpose buffer fit in
-// shared memory): a persistent grid of as many CTAs as the SMs hold.
-template <int LOGK, bool BF16>
-cudaError_t launch_fwht_stream(const void *X, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
+// The streaming kernel for K = 2^LOGK, 11 <= LOGK <= 14: a persistent grid of as many
+// CTAs as the SMs hold.
+template <int LOGK, class Src>
+cudaError_t launch_fwht_stream(const Src &src, int64_t M, const float *gain, float eps, int mode, int8_t *codes,
                                float *scale_x, const ZeroFill &zf, cudaStream_t s) {
-    using S = FwhtShape<LOGK>;
-    using SS = StreamShape<LOGK, BF16>;
-    CUtensorMap tm;
-    if (!make_tmap_rows_3d(&tm, X, BF16, (uint64_t)S::K, (uint64_t)M, (uint32_t)SS::BOX))
-        return cudaErrorInvalidValue;
-    auto kern = act_quant_fwht_stream_kernel<LOGK, BF16>;
+    using S = StreamShape<LOGK>;
+    auto kern = act_quant_fwht_stream_kernel<LOGK, Src>;
     static int bps[kMaxDevices] = {};  // resident CTAs per SM
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int per_sm = dev < kMaxDevices ? bps[dev] : 0;
     if (per_sm == 0) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SS::SMEM);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, S::T, SS::SMEM);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, S::T, S::SMEM);
         if (e != cudaSuccess || per_sm < 1) per_sm = 1;
         if (dev < kMaxDevices) bps[dev] = per_sm;
     }
     const int64_t slots = (int64_t)per_sm * sm_count();
     const int grid = (int)(M < slots ? M : slots);
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(S::T), (size_t)SS::SMEM, s, tm, gain, eps, mode, M, codes,
-                      scale_x, zf, device_status_ptr(), X);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(S::T), (size_t)S::SMEM, s, src, gain, eps, mode, M, codes,
+                      scale_x, zf);
 }
 
 template <int NV8, class Src>
@@ -746,23 +845,17 @@ cudaError_t launch_plain(const Src &src, int64_t M, int K, int T, const float *g
                       codes, scale_x, zf);
 }
 
-// Many tokens of a plain input with 2^11 <= K <= 2^14: the streaming FWHT kernel.
+// Many tokens with 2^11 <= K <= 2^14: the streaming FWHT kernel.
 template <class Src>
-cudaError_t dispatch_stream(const Src &, int64_t, int, const float *, float, int, int8_t *, float *, const ZeroFill &,
-                            cudaStream_t, bool &used) {
-    used = false;
-    return cudaSuccess;
-}
-template <bool BF16>
-cudaError_t dispatch_stream(const XSrc<BF16> &src, int64_t M, int K, const float *gain, float eps, int mode,
+cudaError_t dispatch_stream(const Src &src, int64_t M, int K, const float *gain, float eps, int mode,
                             int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s, bool &used) {
     used = M >= 2 * (int64_t)sm_count();
     if (!used) return cudaSuccess;
     switch (__builtin_ctz((unsigned)K)) {
-        case 11: return launch_fwht_stream<11, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
-        case 12: return launch_fwht_stream<12, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
-        case 13: return launch_fwht_stream<13, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
-        case 14: return launch_fwht_stream<14, BF16>(src.X, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 11: return launch_fwht_stream<11>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 12: return launch_fwht_stream<12>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 13: return launch_fwht_stream<13>(src, M, gain, eps, mode, codes, scale_x, zf, s);
+        case 14: return launch_fwht_stream<14>(src, M, gain, eps, mode, codes, scale_x, zf, s);
         default: used = false; return cudaSuccess;
     }
 }

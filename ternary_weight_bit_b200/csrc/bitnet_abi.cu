@@ -77,20 +77,6 @@ bool make_tmap_out_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t co
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_tmap_rows_3d(CUtensorMap *map, const void *base, bool bf16, uint64_t K, uint64_t M, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn || K % 32 != 0 || box_rows < 1 || box_rows > 256) return false;
-    const uint64_t es = bf16 ? 2 : 4;
-    const cuuint64_t dims[3] = {32, K / 32, M};
-    const cuuint64_t strides[2] = {32 * es, K * es};
-    const cuuint32_t box[3] = {32, box_rows, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base),
-              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int *device_status_ptr() {
     static int *ptrs[kMaxDevices] = {};
     int dev = 0;

@@ -24,11 +24,6 @@ bool make_tmap_u8_2d(CUtensorMap *map, const void *base, uint64_t row_bytes, uin
 bool make_tmap_out_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t cols, uint64_t rows, uint32_t box_x,
                       uint32_t box_y);
 
-// 3D tensor map over a row-major [M][K] fp32 or bf16 activation matrix viewed as
-// [M][K/32][32] (32-element rows of 128 or 64 bytes), box {32, box_rows, 1}, swizzled
-// 128 B (fp32) or 64 B (bf16).  K % 32 == 0 and box_rows <= 256.
-bool make_tmap_rows_3d(CUtensorMap *map, const void *base, bool bf16, uint64_t K, uint64_t M, uint32_t box_rows);
-
 // Per-device address of the library's device status word.
 int *device_status_ptr();
 

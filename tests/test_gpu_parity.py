@@ -108,10 +108,12 @@ def test_act_quant_bf16_and_gain(fwht):
 @pytest.mark.parametrize("K,mode,xdt,gain,M", [
     (2048, "int8", "f32", False, 300), (4096, "int4", "f32", False, 333), (8192, "int8", "bf16", False, 300),
     (16384, "int4", "f32", False, 301), (4096, "int8", "bf16", True, 500), (16384, "int8", "f32", True, 297),
+    (2048, "int4", "bf16", True, 400), (8192, "int4", "f32", True, 1000),
 ])
 def test_act_quant_fwht_streaming(K, mode, xdt, gain, M):
-    # many tokens (M >= 2 x SMs): the persistent FWHT kernel that TMA-loads token rows into
-    # double-buffered swizzled shared memory; every token checked against the oracle
+    # many tokens (M >= 2 x SMs): the persistent FWHT kernel (two register phases around one
+    # swizzled shared-memory transpose, several tokens per CTA); every token checked against
+    # the oracle
     gen = synthetic.generator(K + M)
     X = synthetic.student_t3((M, K), gen)
     X[:, synthetic.outlier_channels(K, K // 100, gen)] *= 50.0
@@ -565,6 +567,8 @@ def _swiglu_case(M, K, N, mode, fwht, xdt, seed, sample_rows=None):
     (13, 1024, 700, "int8", False, "bf16"),  # decode kernel, ragged N, plain quantiser
     (300, 4096, 1000, "int4", True, "f32"),  # tcgen05 kernel, ragged
     (129, 2048, 640, "int8", True, "bf16"),
+    (400, 2048, 512, "int8", True, "bf16"),  # streaming FWHT kernel on the SwiGLU product
+    (300, 16384, 256, "int4", True, "f32"),
 ])
 def test_forward_swiglu(M, K, N, mode, fwht, xdt):
     # silu(gate) * up formed inside the activation kernel (BitNetV2FFN.forward's down projection)
