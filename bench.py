@@ -3,24 +3,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
-A step is one pass of the whole per-token path -- RMSNorm, optional FWHT,
-activation quantisation, ternary GEMM/GEMV, fp32 epilogue -- over one batch of
-the workload (weights are packed once, before timing, as a deployment would).
-The default workload is the largest configuration that fits one GPU: the M = 8192
-point of the 4096-hidden M-sweep, int4 absmean + FWHT, X Student-t(3) with 1 %
-outlier channels x50, against Wo [4096 x 4096] and Wdown [4096 x 16384]; one step
-runs the two forwards (1.37 Tera integer ops).  The same line carries a `decode`
+A pass is the whole per-token path -- RMSNorm, optional FWHT, activation
+quantisation, ternary GEMM/GEMV, fp32 epilogue -- over one batch of the workload
+(weights are packed once, before timing, as a deployment would).  A step is B
+such passes over B batches (the input rotations in turn), B chosen before timing
+so that one step holds at least 5 ms of device work (`config.batches_per_step`):
+even a short run of timed steps then spans tens of clock samples.  The default
+workload is the largest configuration that fits one GPU: the M = 8192 point of the
+4096-hidden M-sweep, int4 absmean + FWHT, X Student-t(3) with 1 % outlier channels
+x50, against Wo [4096 x 4096] and Wdown [4096 x 16384]; one pass runs the two
+forwards (1.37 Tera integer ops).  The same line carries a `decode`
 sub-record: the decode configuration (int8 absmax, no FWHT, M in {1, 4, 8} against
-W [6912 x 2560] and [2560 x 6912], six forwards per step) measured the same way with
+W [6912 x 2560] and [2560 x 6912], six forwards per pass) measured the same way with
 its own roofline, step time and CPU baseline, and a `decode_tl2` sub-record: the same
 decode configuration with the weights in the TL2 format (5 bits per 3 weights).
 Inputs are seeded synthetic tensors.
 
-Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
+Timing: W untimed warm-up steps, then exactly K steps, each one CUDA graph replay,
 bracketed by a barrier and a device synchronisation, timed with CUDA events on the
 launching stream; the maximum over ranks is reported.  Inputs larger than 4x L2
-(the default workload's step reads 691 MiB), or rotated over enough copies that
-every step reads them from HBM.  Clocks are read through NVML every 2 ms during the
+(the default workload's pass reads 691 MiB), or rotated over enough copies that
+every pass reads them from HBM.  Clocks are read through NVML every 2 ms during the
 timed region.  With N > 1 (torchrun), every rank runs its own replica of the
 workload (the path has no cross-GPU exchange); value = tokens of all ranks / max
 rank time.
@@ -61,6 +64,7 @@ METRIC = "ternary GEMM TOPS & weight GB/s vs roofline; H-BitLinear tokens/s (1 B
 # per step.  The default run adds the decode configuration as a sub-record.
 DEFAULT_WORKLOAD = "msweep_M8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+MAX_BATCHES = 512  # passes per timed step at most
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -402,7 +406,8 @@ def _timed_graph_replays(torch, graph, stream, min_s: float, max_reps: int = 100
     return e0.elapsed_time(e1), reps
 
 
-def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sampler, stream, sub_s=0.4, e2e=True):
+def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sampler, stream, sub_s=0.4, e2e=True,
+                    min_step_ms=5.0):
     """One forward workload on this rank: the timed steps (CUDA graphs, events on the
     launching stream), then the dominant kernel alone, the activation kernel alone and
     the end-to-end public call.  Returns the rank-local figures."""
@@ -465,15 +470,36 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
         for i in range(max(1, min(warmup, R))):
             step(i % R)  # eager warm-up also primes the per-device attribute caches
     stream.synchronize()
-    graphs = []
+    # One pass = every case once on one rotation of the inputs.  A timed step is `batches`
+    # passes (rotations in turn) captured in one CUDA graph, enough for MIN_STEP_MS of
+    # device time, so that a few timed steps still span tens of clock samples.
+    ones = []
     for r in range(R):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(r)
-        graphs.append(g)
+        ones.append(g)
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            ones[r].replay()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            ones[r].replay()
+    p1.record(stream)
+    p1.synchronize()
+    pass_ms = max(p0.elapsed_time(p1) / R, 1e-3)
+    batches = int(max(1, min(MAX_BATCHES, math.ceil(min_step_ms / pass_ms))))
+    del ones
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph, stream=stream):
+        for b in range(batches):
+            step(b % R)
     with torch.cuda.stream(stream):
         for i in range(warmup):
-            graphs[i % R].replay()
+            step_graph.replay()
     stream.synchronize()
     assert tb.bitnet_get_last_device_status(stream) == 0
 
@@ -488,7 +514,7 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
     e0.record(stream)
     with torch.cuda.stream(stream):
         for i in range(steps):
-            graphs[i % R].replay()
+            step_graph.replay()
     e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize(dev)
@@ -498,8 +524,8 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
     elapsed = e0.elapsed_time(e1)
     clocks = sampler.summary(t_wall0, t_wall1) if sampler is not None else None
     status = tb.bitnet_get_last_device_status(stream)
-    tokens_rank = steps * sum(c.M for c in host)
-    kernels_per_step = sum(tb.bitnet_forward_kernel_count(c.M, c.N, c.K, c.fwht) for c in host)
+    tokens_rank = steps * batches * sum(c.M for c in host)
+    kernels_per_step = batches * sum(tb.bitnet_forward_kernel_count(c.M, c.N, c.K, c.fwht) for c in host)
 
     # ------------------------------------------------------------------ dominant kernel alone
     peaks, peak_src = load_peaks()
@@ -615,9 +641,8 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
                    "h2d_bytes_per_step": sum(in_bytes(c) for c in host),
                    "d2h_bytes_per_step": sum(out_bytes * c.M * c.N for c in host),
                    "note": "eager calls of the public forward with pinned host inputs in and output out per step"}
-    for g in graphs:
-        del g
-    return {"cases": cases, "host": host, "R": R, "step_bytes": step_bytes, "elapsed_ms": elapsed,
+    del step_graph
+    return {"cases": cases, "host": host, "R": R, "batches": batches, "step_bytes": step_bytes, "elapsed_ms": elapsed,
             "tokens_rank": tokens_rank, "clocks": clocks, "status": status, "roofline": roof,
             "act_quant": act,
             "gemm_tops": round(gemm_ops / (gemm_ms / 1e3) / 1e12, 3),
@@ -649,16 +674,15 @@ def run_ours(args):
     max_ms, tokens_all = aggregate(m["elapsed_ms"], m["tokens_rank"], world, dev)
     sub = sub_tl2 = None
     if args.workload == DEFAULT_WORKLOAD and not args.no_decode_record:
-        # the decode configuration, same rules, in the same process: enough steps for
-        # about half a second of timed work
-        d_steps = max(args.steps, 2000)
+        # the decode configuration, same rules (steps of at least 5 ms), in the same process
+        d_steps = args.steps
         d = measure_forward(torch, tb, "decode", dev, world, d_steps, args.warmup, bf16_out, sampler, stream,
                             e2e=False)
         d_ms, d_tok = aggregate(d["elapsed_ms"], d["tokens_rank"], world, dev)
         sub = {"workload": workload_text("decode"), "name": "decode", "steps": d_steps, "warmup": args.warmup,
                "value": round(d_tok / (d_ms / 1e3), 1), "unit": "tokens/s",
-               "ms_per_step": round(d_ms / d_steps, 6), "roofline": d["roofline"],
-               "act_quant": d["act_quant"], "gpu_launches": d["gpu_launches"],
+               "ms_per_step": round(d_ms / d_steps, 6), "batches_per_step": d["batches"],
+               "roofline": d["roofline"], "act_quant": d["act_quant"], "gpu_launches": d["gpu_launches"],
                "clocks": {k: d["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
                "device_status": d["status"]}
         # the same decode configuration with the weights in the TL2 format
@@ -667,7 +691,8 @@ def run_ours(args):
         t_ms, t_tok = aggregate(t["elapsed_ms"], t["tokens_rank"], world, dev)
         sub_tl2 = {"workload": workload_text("decode_tl2"), "name": "decode_tl2", "steps": d_steps,
                    "value": round(t_tok / (t_ms / 1e3), 1), "unit": "tokens/s",
-                   "ms_per_step": round(t_ms / d_steps, 6), "roofline": t["roofline"],
+                   "ms_per_step": round(t_ms / d_steps, 6), "batches_per_step": t["batches"],
+                   "roofline": t["roofline"],
                    "gpu_launches": t["gpu_launches"], "device_status": t["status"]}
     sampler.stop()
 
@@ -680,6 +705,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": workload_text(args.workload), "name": args.workload,
+                       "batches_per_step": m["batches"],
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} copies ({R * step_bytes / 2**20:.0f} MiB > 4x L2)"
                        if R > 1 else f"per-step working set {step_bytes / 2**20:.0f} MiB, larger than 4x L2",
@@ -983,7 +1009,7 @@ def run_library_int8_probe(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,

@@ -5,10 +5,12 @@
 // quantise), fast_hadamard_transform and Eq. 3/4 (H_m = (1/sqrt2)[[H,H],[H,-H]]),
 // quantize_act_int8 (Eq. 5) and quantize_act_int4 (Eq. 6).
 //
-// One CTA per token; X is read from HBM exactly once (128-bit loads) and the
-// codes are written once.  Everything in between stays on chip.
+// X is read from HBM exactly once and the codes are written once; everything in
+// between stays on chip.  Few tokens: one CTA per token (the plain and the per-token
+// FWHT kernels).  Many tokens with 2^11 <= K <= 2^14: the streaming FWHT kernel, a
+// persistent grid that takes the tokens in turn (described at its definition).
 //
-// FWHT kernel (K = 2^LOGK): each thread owns E = 2^ELOG elements.  The transform
+// Per-token FWHT kernel (K = 2^LOGK): each thread owns E = 2^ELOG elements.  The transform
 // runs as unnormalised radix-2 butterflies (a+b, a-b) over bits 0, 1, ..., LOGK-1
 // in increasing order, in phases of ELOG bits: inside a phase the butterflies are
 // in registers; between phases the token is transposed through shared memory so
@@ -439,7 +441,7 @@ act_quant_fwht_kernel(Src src, const float *__restrict__ gain, float eps, int mo
 // fma(b, -1, a): the same single rounding as a subtraction), except in the register bit
 // that forms the pairs.  The bits are transformed in another order than in the per-token
 // kernel, so results differ from it in the last bits only.  Each token's row is prefetched
-// into L2 two tokens ahead; the barriers per token are two: after the transpose's stores,
+// into L2 one token ahead; the barriers per token are two: after the transpose's stores,
 // and in the statistic's reduction, whose result every thread then finishes itself.
 template <int LOGK>
 struct StreamShape {
@@ -501,7 +503,9 @@ act_quant_fwht_stream_kernel(Src src, const float *__restrict__ gain, float eps,
     pdl_wait_prerequisites();
 
     for (int64_t t = blockIdx.x; t < M; t += gridDim.x) {
-        if (tid == 0 && t + 2 * (int64_t)gridDim.x < M) src.prefetch((t + 2 * (int64_t)gridDim.x) * K, K);
+        // the next token's row: one token ahead keeps the rows in flight (two per CTA) well
+        // inside L2; two ahead overran it at K = 16384 and rows were read from HBM twice
+        if (tid == 0 && t + gridDim.x < M) src.prefetch((t + gridDim.x) * K, K);
         zero_fill(zf, t);  // a following split-K GEMM's output row (and, for token 0, its counters)
         const int64_t row = t * K;
 
@@ -512,13 +516,13 @@ act_quant_fwht_stream_kernel(Src src, const float *__restrict__ gain, float eps,
             v[j].x = src.get1(row + tid + ((2 * j) << TLOG));
             v[j].y = src.get1(row + tid + ((2 * j + 1) << TLOG));
         }
-        float2 sa = make_float2(0.0f, 0.0f), sb = sa;
+        float2 sacc[4];
 #pragma unroll
-        for (int j = 0; j < NP; j += 2) {
-            sa = __ffma2_rn(v[j], v[j], sa);
-            sb = __ffma2_rn(v[j + 1], v[j + 1], sb);
-        }
-        float ss = __fadd_rn(__fadd_rn(sa.x, sa.y), __fadd_rn(sb.x, sb.y));
+        for (int a = 0; a < 4; ++a) sacc[a] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) sacc[j & 3] = __ffma2_rn(v[j], v[j], sacc[j & 3]);
+        const float2 s01 = __fadd2_rn(sacc[0], sacc[1]), s23 = __fadd2_rn(sacc[2], sacc[3]);
+        float ss = __fadd_rn(__fadd_rn(s01.x, s01.y), __fadd_rn(s23.x, s23.y));
         asm volatile("" : "+f"(ss));  // keep the sum here, not sunk to its use after phase 1
         if (gain != nullptr) {
 #pragma unroll
@@ -554,22 +558,23 @@ act_quant_fwht_stream_kernel(Src src, const float *__restrict__ gain, float eps,
 
         // one reduction of (sum x^2, max|z| or sum|z|); every thread finishes it
         float st;
-        if (mean) {
-            float a0 = 0.0f, a1 = 0.0f;
+        {
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four short chains
+            if (mean) {
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                a0 += fabsf(v[j].x);
-                a1 += fabsf(v[j].y);
-            }
-            st = a0 + a1;
-        } else {
-            float a0 = 0.0f, a1 = 0.0f;
+                for (int j = 0; j < NP; ++j) {
+                    acc[2 * (j & 1)] += fabsf(v[j].x);
+                    acc[2 * (j & 1) + 1] += fabsf(v[j].y);
+                }
+                st = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                a0 = fmaxf(a0, fabsf(v[j].x));
-                a1 = fmaxf(a1, fabsf(v[j].y));
+                for (int j = 0; j < NP; ++j) {
+                    acc[2 * (j & 1)] = fmaxf(acc[2 * (j & 1)], fabsf(v[j].x));
+                    acc[2 * (j & 1) + 1] = fmaxf(acc[2 * (j & 1) + 1], fabsf(v[j].y));
+                }
+                st = fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3]));
             }
-            st = fmaxf(a0, a1);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
