@@ -820,15 +820,29 @@ def run_kv(args):
         for i in range(max(1, min(args.warmup, R))):
             step(i % R)
     stream.synchronize()
-    graphs = []
-    for r in range(R):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+    # a timed step is `batches` passes (rotations in turn) in one graph, at least 5 ms
+    one = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(one, stream=stream):
+        for r in range(R):
             step(r)
-        graphs.append(g)
+    with torch.cuda.stream(stream):
+        one.replay()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    with torch.cuda.stream(stream):
+        one.replay()
+    p1.record(stream)
+    p1.synchronize()
+    batches = int(max(1, min(MAX_BATCHES, math.ceil(5.0 / max(p0.elapsed_time(p1) / R, 1e-3)))))
+    del one
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph, stream=stream):
+        for b in range(batches):
+            step(b % R)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs[i % R].replay()
+            step_graph.replay()
     stream.synchronize()
     sampler = clock_sampler(props)
     sampler.start()
@@ -843,7 +857,7 @@ def run_kv(args):
     e0.record(stream)
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            graphs[i % R].replay()
+            step_graph.replay()
     e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize(dev)
@@ -851,7 +865,7 @@ def run_kv(args):
     if world > 1:
         dist.barrier()
     elapsed = e0.elapsed_time(e1)
-    max_ms, tokens_all = aggregate(elapsed, args.steps * B * S, world, dev)
+    max_ms, tokens_all = aggregate(elapsed, args.steps * batches * B * S, world, dev)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
     status = tb.bitnet_get_last_device_status(stream)
@@ -915,7 +929,7 @@ def run_kv(args):
             "metric": METRIC, "value": round(tokens_all / (max_ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": KV_TEXT, "name": "kvcache",
+            "config": {"workload": KV_TEXT, "name": "kvcache", "batches_per_step": batches,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} copies ({R * in_bytes / 2**20:.0f} MiB > 4x L2)",
                        "cuda_graphs": True, "pdl": True},
@@ -924,14 +938,13 @@ def run_kv(args):
                     "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": sum(c.numel() + 4 * s.numel()
                                                                                for c, s in zip(pin_c, pin_s)),
                     "note": "eager bitnet_kv_quant calls with pinned host K, V in and codes, steps out per step"},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 2 * batches * args.steps,
             "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples", "source")},
             "device_status": status,
         }
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-        graphs.clear()
         dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:

@@ -184,9 +184,6 @@ struct SwigluSrc {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = swiglu(v[i], u[i]);
     }
-    __device__ __forceinline__ float get1(int64_t idx) const {
-        return swiglu(load1<BF16>(gate, idx), load1<BF16>(up, idx));
-    }
     __device__ __forceinline__ void get4(int64_t idx, float *v) const {
         float u[4];
         load4<BF16>(gate, idx, v);
@@ -850,9 +847,18 @@ cudaError_t launch_plain(const Src &src, int64_t M, int K, int T, const float *g
                       codes, scale_x, zf);
 }
 
-// Many tokens with 2^11 <= K <= 2^14: the streaming FWHT kernel.
+// Many tokens of a plain input with 2^11 <= K <= 2^14: the streaming FWHT kernel.  The
+// SwiGLU source stays on the per-token kernel: inlined 128 times per thread, its exp and
+// IEEE division made the streaming kernel several times slower (0.11 of HBM on the
+// 2048 x 8192 Wdown input against 0.4 per token).
 template <class Src>
-cudaError_t dispatch_stream(const Src &src, int64_t M, int K, const float *gain, float eps, int mode,
+cudaError_t dispatch_stream(const Src &, int64_t, int, const float *, float, int, int8_t *, float *, const ZeroFill &,
+                            cudaStream_t, bool &used) {
+    used = false;
+    return cudaSuccess;
+}
+template <bool BF16>
+cudaError_t dispatch_stream(const XSrc<BF16> &src, int64_t M, int K, const float *gain, float eps, int mode,
                             int8_t *codes, float *scale_x, const ZeroFill &zf, cudaStream_t s, bool &used) {
     used = M >= 2 * (int64_t)sm_count();
     if (!used) return cudaSuccess;

@@ -567,7 +567,7 @@ def _swiglu_case(M, K, N, mode, fwht, xdt, seed, sample_rows=None):
     (13, 1024, 700, "int8", False, "bf16"),  # decode kernel, ragged N, plain quantiser
     (300, 4096, 1000, "int4", True, "f32"),  # tcgen05 kernel, ragged
     (129, 2048, 640, "int8", True, "bf16"),
-    (400, 2048, 512, "int8", True, "bf16"),  # streaming FWHT kernel on the SwiGLU product
+    (400, 2048, 512, "int8", True, "bf16"),  # many tokens: the per-token FWHT kernel on the SwiGLU product
     (300, 16384, 256, "int4", True, "f32"),
 ])
 def test_forward_swiglu(M, K, N, mode, fwht, xdt):
