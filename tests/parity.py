@@ -18,6 +18,7 @@ Rules (from the BitNet v2 page's Eq. 5/6 and the exactness of integer arithmetic
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 
@@ -38,12 +39,17 @@ def check_codes(gpu: np.ndarray, ora: np.ndarray, shadow: np.ndarray, label: str
     d = gpu - ora
     flips = np.nonzero(d)
     nflip = len(flips[0])
+    worst = 0.0
     if nflip:
         assert np.abs(d).max() == 1, f"{label}: a code differs by {np.abs(d).max()}"
         boundary = (gpu[flips] + ora[flips]) / 2.0
         dist = np.abs(shadow[flips] - boundary)
         worst = float(dist.max())
         assert worst <= TIE_TOL, f"{label}: a flipped code is {worst:.3g} code units from its rounding tie"
+    log = os.environ.get("BITNET_PARITY_LOG")  # optional record of every comparison: label, codes, flips, worst
+    if log:
+        with open(log, "a") as f:
+            f.write(f"{label}\t{gpu.size}\t{nflip}\t{worst:.3e}\n")
     allowed = max(1, int(math.floor(FLIP_RATE * gpu.size)))
     assert nflip <= allowed, f"{label}: {nflip} flipped codes of {gpu.size} (allowed {allowed})"
     return nflip
