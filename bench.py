@@ -22,8 +22,9 @@ Inputs are seeded synthetic tensors.
 Timing: W untimed warm-up steps, then exactly K steps, each one CUDA graph replay,
 bracketed by a barrier and a device synchronisation, timed with CUDA events on the
 launching stream; the maximum over ranks is reported.  Inputs larger than 4x L2
-(the default workload's pass reads 691 MiB), or rotated over enough copies that
-every pass reads them from HBM.  Clocks are read through NVML every 2 ms during the
+(the default workload's pass reads 660 MiB of X and packed weights), or rotated over
+enough copies that every pass reads them from HBM.  Clocks are read through NVML every
+2 ms during the
 timed region.  With N > 1 (torchrun), every rank runs its own replica of the
 workload (the path has no cross-GPU exchange); value = tokens of all ranks / max
 rank time.
@@ -708,7 +709,7 @@ def run_ours(args):
                        "batches_per_step": m["batches"],
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"inputs rotate over {R} copies ({R * step_bytes / 2**20:.0f} MiB > 4x L2)"
-                       if R > 1 else f"per-step working set {step_bytes / 2**20:.0f} MiB, larger than 4x L2",
+                       if R > 1 else f"per-pass working set {step_bytes / 2**20:.0f} MiB, larger than 4x L2",
                        "cuda_graphs": True, "pdl": True, "out_dtype": args.out_dtype},
             "roofline": m["roofline"],
             "act_quant": m["act_quant"],
