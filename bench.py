@@ -24,8 +24,7 @@ bracketed by a barrier and a device synchronisation, timed with CUDA events on t
 launching stream; the maximum over ranks is reported.  Inputs larger than 4x L2
 (the default workload's pass reads 660 MiB of X and packed weights), or rotated over
 enough copies that every pass reads them from HBM.  Clocks are read through NVML every
-2 ms during the
-timed region.  With N > 1 (torchrun), every rank runs its own replica of the
+2 ms during the timed region.  With N > 1 (torchrun), every rank runs its own replica of the
 workload (the path has no cross-GPU exchange); value = tokens of all ranks / max
 rank time.
 
