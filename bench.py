@@ -382,6 +382,11 @@ def time_oracle(cases, budget_s: float, steps: int | None = None, bf16_out: bool
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def batches_per_step(pass_ms: float, min_step_ms: float) -> int:
+    """Passes per timed step: enough for min_step_ms of device time, 1..MAX_BATCHES."""
+    return int(max(1, min(MAX_BATCHES, math.ceil(min_step_ms / max(pass_ms, 1e-3)))))
+
+
 def _timed_graph_replays(torch, graph, stream, min_s: float, max_reps: int = 100000):
     """Replay `graph` on `stream` for at least min_s seconds (3 untimed replays first);
     returns (milliseconds, replays), timed with CUDA events on that stream."""
@@ -490,8 +495,7 @@ def measure_forward(torch, tb, name, dev, world, steps, warmup, bf16_out, sample
             ones[r].replay()
     p1.record(stream)
     p1.synchronize()
-    pass_ms = max(p0.elapsed_time(p1) / R, 1e-3)
-    batches = int(max(1, min(MAX_BATCHES, math.ceil(min_step_ms / pass_ms))))
+    batches = batches_per_step(p0.elapsed_time(p1) / R, min_step_ms)
     del ones
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph, stream=stream):
@@ -834,7 +838,7 @@ def run_kv(args):
         one.replay()
     p1.record(stream)
     p1.synchronize()
-    batches = int(max(1, min(MAX_BATCHES, math.ceil(5.0 / max(p0.elapsed_time(p1) / R, 1e-3)))))
+    batches = batches_per_step(p0.elapsed_time(p1) / R, 5.0)
     del one
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph, stream=stream):

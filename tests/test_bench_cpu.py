@@ -37,3 +37,28 @@ def test_oracle_sample_is_bounded_and_extrapolated():
     assert "extrapolated" in desc and "tokens" in desc
     rate_bf16, _, _, _ = bench.time_oracle(cases, budget_s=0.5, steps=2, bf16_out=True)
     assert rate_bf16 > 0
+
+
+def test_batches_per_step_spans_the_minimum_step():
+    assert bench.batches_per_step(0.66, 5.0) == 8        # default workload: 8 passes of 0.66 ms
+    assert bench.batches_per_step(0.035, 5.0) == 143     # decode: 143 passes of 35 us
+    assert bench.batches_per_step(7.0, 5.0) == 1         # a pass longer than the minimum
+    assert bench.batches_per_step(0.0, 5.0) == bench.MAX_BATCHES  # no pass time measured: capped
+    for pass_ms in (0.011, 0.2, 1.3, 4.9):
+        b = bench.batches_per_step(pass_ms, 5.0)
+        assert b * pass_ms >= 5.0 or b == bench.MAX_BATCHES
+        assert (b - 1) * pass_ms < 5.0
+
+
+def test_workloads_satisfy_the_boundary_rules():
+    # every bench case passes the ABI's shape rules: K % 128 == 0, K <= 32768, FWHT needs a
+    # power-of-two K, and the decode workloads stay on the GEMV (M <= 16)
+    for name in ("decode", "decode_tl2", "prefill", "wdown", "wdown_swiglu", "msweep_M8", "msweep_M64",
+                 "msweep_M512", "msweep_M4096", "msweep_M8192"):
+        for (label, M, N, K, mode, fwht, xk, xdt, outl) in bench.workload_cases(name):
+            assert K % 128 == 0 and K <= 32768, (name, label)
+            assert not fwht or (K & (K - 1)) == 0, (name, label)
+            assert mode in ("int8", "int4") and xdt in ("f32", "bf16") and M >= 1 and N >= 1
+            if name.startswith("decode"):
+                assert M <= 16
+    assert bench.workload_cases(bench.DEFAULT_WORKLOAD) == bench.workload_cases("msweep_M8192")
